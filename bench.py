@@ -1,0 +1,381 @@
+"""Benchmark: fused RoPE + packed varlen joint attention forward, TFLOP/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload max] [--impl ours|reference]
+
+One step = one h3_varlen_attn_fwd call over the whole packed workload
+(rotary pass over k, then the attention kernel, which rotates each query tile
+as it loads it). FLOPs = sum over segments of 4 L^2 H D (QK^T and PV,
+non-causal). Inputs are seeded synthetic bf16 tensors shaped like the
+workload (each larger than L2, so no flush is needed between steps).
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own packed
+workload (different seed) with no data-path collective: weak scaling. The
+only collectives are the barrier and the max over ranks of the timed region.
+
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the
+same workload (the reference arm); under torchrun only rank 0 runs it.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "fused RoPE+varlen joint attention fwd TFLOP/s and % of B200 BF16 peak"
+UNIT = "TFLOP/s"
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+KERNEL_SOURCES = ["audio_diffusion_transformer_h3_b200/csrc/attn_fwd.cuh",
+                  "audio_diffusion_transformer_h3_b200/csrc/sm100.cuh",
+                  "audio_diffusion_transformer_h3_b200/csrc/rope.cuh"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"bf16": float(d["bf16_tflops"]), "bf16_sustained": float(d["bf16_tflops_sustained"]),
+                "hbm": float(d["hbm_gbs"]), "source": "measured"}
+    return {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, or None
+    if the summary is missing or was taken on a different kernel source."""
+    p = os.path.join(PROFILE_DIR, f"attn_fwd_{workload}_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self) -> dict:
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sms.append(float(f[1]))
+                maxs.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+def workload_config(wl) -> dict:
+    return {"workload": wl.name, "description": wl.description, "tokens": wl.n_tokens,
+            "segments": wl.seg_lens, "heads": wl.heads, "head_dim": wl.head_dim,
+            "rope_split": list(wl.split), "theta": wl.theta, "causal": False,
+            "l2": "each input tensor exceeds the 126 MB L2; no flush between steps"
+            if wl.n_tokens * wl.heads * wl.head_dim * 2 > 126e6 else
+            "L2 flushed (256 MB write) before every timed step"}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def cpu_oracle_sample(wl, q, k, v, pos, cu, budget_s: float):
+    """Time the float64 oracle on (head, 128-row block) units of the workload
+    until ``budget_s`` seconds are spent. Returns (TFLOP/s, description, threads)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    rng = np.random.default_rng(7)
+    flops = 0.0
+    units = 0
+    t0 = time.perf_counter()
+    while True:
+        s = int(rng.integers(0, len(cu) - 1))
+        a, e = int(cu[s]), int(cu[s + 1])
+        h = int(rng.integers(0, wl.heads))
+        r0 = int(rng.integers(a, max(a + 1, e - 128)))
+        rows = np.arange(r0, min(e, r0 + 128))
+        oracle.attention_rows_ref(q, k, v, cu, wl.softmax_scale, rows, [h], pos, wl.split, wl.theta)
+        flops += 4.0 * len(rows) * (e - a) * wl.head_dim
+        units += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    desc = (f"{units} units of (1 head, up to 128 query rows) against their full segment, "
+            f"random over the workload's segments and heads; {flops:.3g} FLOP in {dt:.1f} s")
+    return flops / dt / 1e12, desc, threads
+
+
+# -------------------------------------------------------------------- arms
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return 0
+    q, k, v = synth.draw_qkv(wl)
+    import oracle
+    pos = oracle.packed_positions(wl.segments)
+    cu = synth.cu_seqlens_of(wl.seg_lens)
+    budget = min(args.ref_step_seconds, max(1.0, 90.0 / (args.steps + args.warmup / 4.0)))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(wl, q, k, v, pos, cu, budget / 4)
+    vals = []
+    desc, threads = "", 1
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        val, desc, threads = cpu_oracle_sample(wl, q, k, v, pos, cu, budget)
+        vals.append(val)
+    total = time.perf_counter() - t0
+    value = float(np.mean(vals))
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded, bf16 inputs widened to float64)",
+            "config": workload_config(wl), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, wl, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import audio_diffusion_transformer_h3_b200 as h3
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    seed = wl.the_seed + 7919 * rank
+    q, k, v = synth.draw_qkv(wl, seed=seed)
+    pos, cu = h3.h3_build_positions(wl.segments)
+    N, H, D = wl.n_tokens, wl.heads, wl.head_dim
+    nseg = len(wl.seg_lens)
+    flops_step = wl.flops()
+
+    def pinned_bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+    hq, hk, hv = pinned_bf16(q), pinned_bf16(k), pinned_bf16(v)
+    hpos = torch.from_numpy(pos).pin_memory()
+    hcu = torch.from_numpy(cu).pin_memory()
+    ho = torch.empty((N, H, D), dtype=torch.bfloat16).pin_memory()
+    del q, k, v
+
+    dq, dk, dv = hq.to(dev), hk.to(dev), hv.to(dev)
+    dpos, dcu = hpos.to(dev), hcu.to(dev)
+    do = torch.empty_like(dq)
+    ws = h3.workspace_for(N, H, D, nseg, dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = None
+    if N * H * D * 2 <= 126e6:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        if flush is not None:
+            flush.zero_()
+        h3.varlen_attn_fwd_t(dq, dk, dv, dcu, wl.max_seqlen, dpos, wl.split, wl.theta,
+                             wl.softmax_scale, out=do, workspace=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = h3.device_status_t(ws)
+    if st != h3.H3_OK:
+        raise RuntimeError(f"device status {h3.h3_status_string(st)}")
+
+    # ---- device-timed region: inputs resident in HBM ----
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    barrier()
+    torch.cuda.synchronize()
+    visible = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    smi_id = visible[local_rank] if local_rank < len(visible) else str(local_rank)
+    with ClockSampler(smi_id) as clk:
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]))
+    if h3.device_status_t(ws) != h3.H3_OK:
+        raise RuntimeError("device status not ok after timed region")
+    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    mean_step_ms = float(np.mean(step_ms))
+
+    # ---- end-to-end through the public API with host buffers ----
+    h2d = hq.numel() * 2 * 3 + hpos.numel() * 4 + hcu.numel() * 4
+    d2h = ho.numel() * 2
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dpos.copy_(hpos, non_blocking=True)
+        dcu.copy_(hcu, non_blocking=True)
+        h3.varlen_attn_fwd_t(dq, dk, dv, dcu, wl.max_seqlen, dpos, wl.split, wl.theta,
+                             wl.softmax_scale, out=do, workspace=ws, stream=stream)
+        ho.copy_(do, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = world * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12
+
+    peaks = measured_peaks()
+    achieved = flops_step / (mean_step_ms * 1e-3) / 1e12
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded bf16 ~N(0,1) q/k/v, fp32 positions on the shared clock)",
+        "config": workload_config(wl),
+        "pct_of_bf16_peak": {"burst_measured": 100 * achieved / peaks["bf16"],
+                             "sustained_measured": 100 * achieved / peaks["bf16_sustained"],
+                             "datasheet_2250": 100 * achieved / 2250.0},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16"],
+                     "peak_kind": f"bf16 dense, burst ({peaks['source']})",
+                     "traffic": recorded_traffic(wl.name),
+                     "kernel": "attn_fwd_kernel<128> (step = k rotary pass + attention kernel)"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle  # CPU baseline leg only
+        def host_bits(t):
+            return t.view(torch.int16).numpy().view(np.uint16)
+        opos = oracle.packed_positions(wl.segments)
+        val, desc, threads = cpu_oracle_sample(wl, host_bits(hq), host_bits(hk), host_bits(hv),
+                                               opos, cu, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="max")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = synth.workload(args.workload)
+
+    if args.impl == "reference":
+        return run_reference(args, wl, rank, world)
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,165 @@
+/*
+ * h3attn -- packed variable-length joint video+audio self-attention with a
+ * 3-axis (t, h, w) rotary embedding on the shared audio/video clock, for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What is computed (sources are the public pages on MiniMax-H3):
+ *   - "Day 0 Support for MiniMax-H3 on AMD Instinct GPUs", section "The
+ *     diffusion transformer (DiT)": the DiT flattens the video latent and the
+ *     audio latent into one token sequence and attends over it jointly; its
+ *     position encoding is Rotary (RoPE); heads are 128 wide.
+ *   - "MiniMax H3" vLLM-Omni recipe, section "Step execution and continuous
+ *     batching": co-batched requests are packed into one sequence that keeps
+ *     one attention document per request (a block-diagonal mask given by
+ *     cu_seqlens); section "Attention Backends": packed varlen backends.
+ *   - "MiniMax-H3 Reference" Space README, section "References": the order of
+ *     the references advances the shared audio/video rotary clock.
+ *   - "MiniMax H3 on Moore Threads MUSA", section "MUSA validation": position
+ *     metadata is FP64 on the host and is cast to FP32 before device
+ *     arithmetic.
+ *
+ * Conventions for every call:
+ *   - Tensors q, k, v, o are bf16, layout [N, H, D] ("THD"), contiguous, token
+ *     stride H*D elements. N = total packed tokens, H = heads, D = head dim.
+ *   - pos is fp32 [N, 3] = (t, h, w) per token, contiguous.
+ *   - cu_seqlens is int32 [nseg + 1]: cu[0] = 0, non-decreasing, cu[nseg] = N.
+ *     Segment s holds tokens [cu[s], cu[s+1]); zero-length segments are legal.
+ *   - The caller owns every buffer. No call allocates device memory, and no
+ *     call synchronises the stream except h3_read_device_status.
+ *   - Device calls are asynchronous on `stream` and report argument errors
+ *     through the return value before anything is enqueued. Errors never
+ *     abort or throw across this boundary.
+ *   - Device pointers must point to memory of the current CUDA device.
+ */
+#ifndef H3ATTN_H
+#define H3ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. NULL is the legacy default stream. */
+typedef struct CUstream_st *h3_stream_t;
+
+typedef enum h3_status {
+    H3_OK = 0,
+    H3_ERR_INVALID_ARG = 1,    /* null pointer, bad size, bad rotary split */
+    H3_ERR_UNSUPPORTED = 2,    /* head dim other than 64 or 128, no sm_100 device */
+    H3_ERR_MISALIGNED = 3,     /* q/k/v/o/x/out not 16-byte aligned, pos/lse not 4-byte aligned */
+    H3_ERR_WORKSPACE = 4,      /* workspace null or smaller than h3_workspace_size() */
+    H3_ERR_CUDA = 5,           /* a CUDA runtime/driver call failed; see h3_last_cuda_error() */
+    H3_ERR_DEVICE_TIMEOUT = 6, /* a bounded in-kernel wait gave up (device status only) */
+    H3_ERR_BAD_SEQLENS = 7     /* cu_seqlens invalid on the device (device status only) */
+} h3_status;
+
+/* Rotary split of the head dimension into contiguous (t, h, w) chunks.
+ * Each width is even and d_t + d_h + d_w = D. Inside the chunk of axis a
+ * (width d_a, first channel c_a), pair j (j < d_a/2) is channels
+ * (c_a + 2j, c_a + 2j + 1) and is rotated by the angle
+ * pos[a] * theta^(-2j/d_a):  (x0, x1) -> (x0 cos - x1 sin, x0 sin + x1 cos).
+ * The inverse frequencies are formed in double on the host and rounded to
+ * float; angles, cos and sin are fp32 on the device. */
+typedef struct h3_rope_cfg {
+    int32_t d_t, d_h, d_w;
+    float theta;
+} h3_rope_cfg;
+
+/* Composition of one packed segment (one attention document), in token
+ * order: `image_refs` single-frame reference grids of image_h x image_w
+ * tokens, then `audio_refs` audio-reference runs of audio_ref_len tokens,
+ * then the video latent grid video_t x video_h x video_w (row-major t, h, w),
+ * then `audio_tail` audio tokens spread over the video grid's frames.
+ * Source: "MiniMax-H3 Reference" Space README, sections "References" and
+ * "AoTI-compiled blocks" (reference rows packed in front of generated rows,
+ * their order advancing the shared clock). */
+typedef struct h3_segment_layout {
+    int32_t image_refs, image_h, image_w;
+    int32_t audio_refs, audio_ref_len, audio_rate; /* audio_rate: tokens per clock unit */
+    int32_t video_t, video_h, video_w;
+    int32_t audio_tail;
+} h3_segment_layout;
+
+/* Number of tokens of one segment layout, or -1 if a field is negative or
+ * the count overflows int32. Host only. */
+int64_t h3_segment_tokens(const h3_segment_layout *seg);
+
+/* Host-side position build for `nseg` packed segments (host memory only,
+ * no CUDA call). Writes pos[n] = (t, h, w) as float for every token and, if
+ * cu_seqlens is not NULL, the nseg+1 segment boundaries. Each segment's clock
+ * starts at t0 = 0. Image reference: tokens (t0, h, w), then t0 += 1. Audio
+ * reference: token i at (t0 + i/audio_rate, 0, 0), then
+ * t0 += audio_ref_len/audio_rate. Video grid: (t0 + tau, h, w). Audio tail
+ * token i of n: (t0 + (i*video_t)/n, 0, 0). Every value is formed in double
+ * in the order written and rounded once to float ("MiniMax H3 on Moore
+ * Threads MUSA", section "MUSA validation").
+ * pos: host float [capacity, 3]. Returns H3_ERR_INVALID_ARG on a null
+ * pointer, a bad layout (negative field, audio_rate <= 0 with audio refs) or
+ * if the total exceeds `capacity`. */
+h3_status h3_build_positions(const h3_segment_layout *segs, int32_t nseg, float *pos,
+                             int64_t capacity, int32_t *cu_seqlens);
+
+/* Standalone rotary pass: out = RoPE(x, pos). "Day 0 Support for MiniMax-H3
+ * on AMD Instinct GPUs", section "The diffusion transformer (DiT)".
+ *   x, out : device bf16 [N, H, D], 16-byte aligned; out may equal x
+ *            (in place); other overlap is undefined.
+ *   pos    : device fp32 [N, 3], 4-byte aligned.
+ *   N >= 0 (N = 0 is a no-op), 1 <= H, D in {64, 128}, H*D*N < 2^40.
+ * Results are rounded to bf16 (round to nearest even). Bit-identical to the
+ * rotation that h3_varlen_attn_fwd applies to q and k. One kernel launch. */
+h3_status h3_rope_apply(const void *x, void *out, const float *pos, int64_t N, int32_t H,
+                        int32_t D, h3_rope_cfg rope, h3_stream_t stream);
+
+/* Bytes of device workspace h3_varlen_attn_fwd needs: a 256-byte status
+ * block plus, for the rotated keys, N*H*D*2 bytes rounded up to 256. */
+size_t h3_workspace_size(int64_t N, int32_t H, int32_t D, int32_t nseg);
+
+/* Fused RoPE + packed varlen joint attention, forward, non-causal.
+ * For every segment s and head h, with Q~ = RoPE(q), K~ = RoPE(k) when pos is
+ * not NULL (else Q~ = q, K~ = k):
+ *     O = softmax(softmax_scale * Q~ K~^T) V     over the segment's rows only,
+ *     LSE = row log-sum-exp of softmax_scale * Q~ K~^T (natural log).
+ * Sources: see the file header (joint sequence, RoPE, packed documents).
+ *   q, k, v    : device bf16 [N, H, D], 16-byte aligned, unrotated.
+ *   o          : device bf16 [N, H, D], 16-byte aligned; must not overlap inputs.
+ *   lse        : device fp32 [H, N] or NULL (not written).
+ *   cu_seqlens : device int32 [nseg + 1]; validated on the device: a
+ *                violation (cu[0] != 0, decreasing, cu[nseg] != N, or a
+ *                segment longer than max_seqlen) makes the kernel skip the
+ *                work and set H3_ERR_BAD_SEQLENS in the workspace status.
+ *   max_seqlen : upper bound on every segment length, 1 <= max_seqlen <= N.
+ *   pos        : device fp32 [N, 3] or NULL (no rotary embedding).
+ *   N, H, D    : 0 <= N < 2^31 (N = 0 is a no-op), 1 <= H <= 65535,
+ *                D in {64, 128}; 1 <= nseg <= 65535.
+ *   softmax_scale : finite, >= 0 (0 gives the mean of V over the segment).
+ *   workspace  : device, 256-byte aligned, >= h3_workspace_size(N, H, D, nseg)
+ *                bytes; owned by the caller, must not be shared by calls that
+ *                run concurrently. Its status word is reset by every call.
+ * Accumulation is fp32; P is rounded to bf16 before the PV product; O is
+ * rounded to bf16. Results are deterministic run to run. Launches: one
+ * rotary kernel for k (when pos is not NULL) and one attention kernel. */
+h3_status h3_varlen_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                             const int32_t *cu_seqlens, int32_t nseg, int32_t max_seqlen,
+                             const float *pos, h3_rope_cfg rope, int64_t N, int32_t H,
+                             int32_t D, float softmax_scale, void *workspace,
+                             size_t workspace_bytes, h3_stream_t stream);
+
+/* Waits for `stream`, then returns the device status word of the last call
+ * that used `workspace` (H3_OK, H3_ERR_BAD_SEQLENS or H3_ERR_DEVICE_TIMEOUT),
+ * or H3_ERR_CUDA if the copy fails. */
+h3_status h3_read_device_status(const void *workspace, h3_stream_t stream);
+
+/* Static description of a status code. Never NULL. */
+const char *h3_status_string(h3_status status);
+
+/* cudaError_t value of the most recent H3_ERR_CUDA on the calling thread
+ * (0 if none). */
+int32_t h3_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* H3ATTN_H */

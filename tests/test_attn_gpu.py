@@ -1,0 +1,234 @@
+"""h3_varlen_attn_fwd on the GPU against the float64 oracle.
+
+Tolerance (bf16 in, fp32 accumulate, bf16 out): max |gpu - oracle| <= 2e-2
+and mean |gpu - oracle| <= 2e-3 over the compared elements; every output is
+finite. Small workloads are compared in full; the large ones, in the launch
+configuration the benchmark times, on sampled rows that the oracle computes
+one by one, plus properties that hold at any size.
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import MAX_ABS, MEAN_ABS, assert_close_bf16, dev, dev_bf16, host_bits, host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _h3():
+    import audio_diffusion_transformer_h3_b200 as h3
+    return h3
+
+
+def _run(q, k, v, cu, max_seqlen, pos, split, scale, return_lse=True, theta=1e4):
+    import torch
+    h3 = _h3()
+    tq, tk, tv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    tcu = dev(np.asarray(cu, dtype=np.int32))
+    tp = dev(pos) if pos is not None else None
+    N, H, D = q.shape
+    ws = h3.workspace_for(N, H, D, len(cu) - 1)
+    out = h3.varlen_attn_fwd_t(tq, tk, tv, tcu, max_seqlen, tp, split, theta, scale,
+                               return_lse=return_lse, workspace=ws)
+    torch.cuda.synchronize()
+    assert h3.device_status_t(ws) == h3.H3_OK
+    return out
+
+
+def _case(seg_lens, H, D, split, seed, pos_range=64.0):
+    q, k, v, pos, cu = synth.draw_random_case(seg_lens, H, D, seed, pos_range=pos_range)
+    return q, k, v, pos, cu, split
+
+
+# ------------------------------------------------------------ full parity
+
+def test_tiny_workload_full_parity():
+    wl = synth.workload("tiny")
+    q, k, v = synth.draw_qkv(wl)
+    pos = oracle.packed_positions(wl.segments)
+    cu = synth.cu_seqlens_of(wl.seg_lens)
+    o, lse = _run(q, k, v, cu, wl.max_seqlen, pos, wl.split, wl.softmax_scale)
+    O, L = oracle.attention_ref(q, k, v, cu, wl.softmax_scale, pos, wl.split)
+    assert_close_bf16(host_f64(o), O, "tiny")
+    np.testing.assert_allclose(host_f64(lse), L, rtol=0, atol=1e-2)
+
+
+@pytest.mark.parametrize("D,split", [(64, (16, 24, 24)), (128, (32, 48, 48))])
+@pytest.mark.parametrize("seg_lens", [
+    [1], [2], [63], [64], [65], [127], [128], [129], [255], [256], [257], [300],
+    [1, 2, 63, 64, 65, 127, 128, 129],             # non-128-aligned segment starts
+    [0, 200, 0, 0, 77, 0],                        # zero-length segments
+    [513, 1, 384, 700],
+])
+def test_edge_segments_full_parity(seg_lens, D, split):
+    H = 3
+    q, k, v, pos, cu, split = _case(seg_lens, H, D, split, seed=sum(seg_lens) + D)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = _run(q, k, v, cu, max(max(seg_lens), 1), pos, split, scale)
+    O, L = oracle.attention_ref(q, k, v, cu, scale, pos, split)
+    assert_close_bf16(host_f64(o), O, f"segments {seg_lens} D={D}")
+    np.testing.assert_allclose(host_f64(lse), L, rtol=0, atol=1e-2)
+
+
+def test_no_rope_and_scale_variants():
+    q, k, v, pos, cu, split = _case([100, 260], 2, 128, (32, 48, 48), seed=21)
+    for scale in (0.0, 0.05, 1.0 / math.sqrt(128), 0.3):
+        o, lse = _run(q, k, v, cu, 260, None, None, scale)
+        O, L = oracle.attention_ref(q, k, v, cu, scale)
+        assert_close_bf16(host_f64(o), O, f"no rope, scale {scale}")
+
+
+def test_single_workload_sampled_all_heads():
+    wl = synth.workload("single")
+    q, k, v = synth.draw_qkv(wl)
+    pos = oracle.packed_positions(wl.segments)
+    cu = synth.cu_seqlens_of(wl.seg_lens)
+    o, lse = _run(q, k, v, cu, wl.max_seqlen, pos, wl.split, wl.softmax_scale)
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.r_[0:130, 8000:8320, rng.integers(0, wl.n_tokens, 300)])
+    heads = list(range(wl.heads))
+    O, L = oracle.attention_rows_ref(q, k, v, cu, wl.softmax_scale, rows, heads, pos, wl.split)
+    assert_close_bf16(host_f64(o)[rows], O, "single")
+    np.testing.assert_allclose(host_f64(lse)[:, rows], L, rtol=0, atol=1e-2)
+
+
+# ----------------------------------------- full-size workloads, sampled rows
+
+def _sample_rows(cu, rng, per_seg=48):
+    rows = []
+    for s in range(len(cu) - 1):
+        a, e = int(cu[s]), int(cu[s + 1])
+        cand = [a, a + 1, a + 127, a + 128, a + 129, a + 255, a + 256, e - 129, e - 128,
+                e - 2, e - 1]
+        rows += [r for r in cand if a <= r < e]
+        rows += list(rng.integers(a, e, per_seg))
+    return np.unique(np.asarray(rows, dtype=np.int64))
+
+
+@pytest.mark.parametrize("name", ["long", "packed", "max"])
+def test_large_workloads_sampled_parity_and_properties(name):
+    import torch
+    wl = synth.workload(name)
+    q, k, v = synth.draw_qkv(wl)
+    pos = oracle.packed_positions(wl.segments)
+    cu = synth.cu_seqlens_of(wl.seg_lens)
+    o, lse = _run(q, k, v, cu, wl.max_seqlen, pos, wl.split, wl.softmax_scale)
+    rng = np.random.default_rng(wl.index)
+    rows = _sample_rows(cu, rng)
+    heads = sorted({0, wl.heads // 2, wl.heads - 1, int(rng.integers(0, wl.heads))})
+    O, L = oracle.attention_rows_ref(q, k, v, cu, wl.softmax_scale, rows, heads, pos, wl.split)
+    got = host_f64(o[torch.as_tensor(rows).cuda()][:, heads])
+    assert_close_bf16(got, O, name)
+    np.testing.assert_allclose(host_f64(lse[heads][:, torch.as_tensor(rows).cuda()]), L,
+                               rtol=0, atol=1e-2)
+    # every output is finite and, as a convex combination of its segment's V
+    # rows, lies inside their per-channel range
+    assert bool(torch.isfinite(o.float()).all())
+    tv = dev_bf16(v).float()
+    of = o.float()
+    for s in range(len(cu) - 1):
+        a, e = int(cu[s]), int(cu[s + 1])
+        lo = tv[a:e].amin(0, keepdim=True) - 1e-2
+        hi = tv[a:e].amax(0, keepdim=True) + 1e-2
+        assert bool(((of[a:e] >= lo) & (of[a:e] <= hi)).all())
+
+
+# ------------------------------------------------------------- invariants
+
+def test_packed_equals_alone_bitwise():
+    seg_lens = [300, 129, 1000, 64]
+    q, k, v, pos, cu, split = _case(seg_lens, 2, 128, (32, 48, 48), seed=31)
+    o = _run(q, k, v, cu, 1000, pos, split, 0.09, return_lse=False)
+    ob = host_bits(o)
+    for s in range(len(seg_lens)):
+        a, e = cu[s], cu[s + 1]
+        os_ = _run(q[a:e], k[a:e], v[a:e], np.array([0, e - a], np.int32), e - a, pos[a:e],
+                   split, 0.09, return_lse=False)
+        assert np.array_equal(host_bits(os_), ob[a:e]), s
+
+
+def test_fused_rope_equals_prerotated_inputs_bitwise():
+    import torch
+    h3 = _h3()
+    q, k, v, pos, cu, split = _case([700, 333], 4, 128, (32, 48, 48), seed=41)
+    o1 = _run(q, k, v, cu, 700, pos, split, 0.1, return_lse=False)
+    tq = h3.rope_apply_t(dev_bf16(q), dev(pos), split)
+    tk = h3.rope_apply_t(dev_bf16(k), dev(pos), split)
+    torch.cuda.synchronize()
+    o2 = _run(host_bits(tq), host_bits(tk), v, cu, 700, None, None, 0.1, return_lse=False)
+    assert np.array_equal(host_bits(o1), host_bits(o2))
+
+
+def test_deterministic_run_to_run():
+    q, k, v, pos, cu, split = _case([900, 2000], 3, 128, (32, 48, 48), seed=51)
+    a = _run(q, k, v, cu, 2000, pos, split, 0.08)
+    b = _run(q, k, v, cu, 2000, pos, split, 0.08)
+    assert np.array_equal(host_bits(a[0]), host_bits(b[0]))
+    assert np.array_equal(a[1].cpu().numpy().view(np.uint32), b[1].cpu().numpy().view(np.uint32))
+
+
+def test_single_token_segments_return_v_exactly():
+    q, k, v, pos, cu, split = _case([1] * 37, 2, 64, (16, 24, 24), seed=61)
+    o = _run(q, k, v, cu, 1, pos, split, 0.125, return_lse=False)
+    assert np.array_equal(host_bits(o), v)
+
+
+def test_uniform_scores_give_segment_mean():
+    q, k, v, pos, cu, split = _case([90, 400], 2, 128, (32, 48, 48), seed=71)
+    o = _run(np.zeros_like(q), k, v, cu, 400, pos, split, 0.1, return_lse=False)
+    V = oracle.bf16_bits_to_f64(v)
+    got = host_f64(o)
+    for s in range(2):
+        a, e = cu[s], cu[s + 1]
+        assert_close_bf16(got[a:e], np.broadcast_to(V[a:e].mean(0), got[a:e].shape), "mean")
+
+
+def test_skewed_keys_large_logits():
+    # keys offset by a large per-head constant: the running max moves a lot
+    q, k, v, pos, cu, split = _case([1500], 2, 128, (32, 48, 48), seed=81)
+    kk = oracle.bf16_bits_to_f64(k)
+    kk[:, 0, :] += 3.0
+    kk[700:, 1, :] += 6.0
+    kb = synth.f32_to_bf16_bits(kk.astype(np.float32))
+    o, lse = _run(q, kb, v, cu, 1500, pos, split, 1.0 / math.sqrt(128))
+    O, L = oracle.attention_ref(q, kb, v, cu, 1.0 / math.sqrt(128), pos, split)
+    assert_close_bf16(host_f64(o), O, "skewed")
+    np.testing.assert_allclose(host_f64(lse), L, rtol=0, atol=2e-2)
+
+
+# ------------------------------------------------------------- error paths
+
+def test_bad_cu_seqlens_sets_device_status_without_fault():
+    import torch
+    h3 = _h3()
+    q, k, v, pos, cu, split = _case([100, 100], 2, 64, (16, 24, 24), seed=91)
+    tq, tk, tv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    ws = h3.workspace_for(200, 2, 64, 2)
+    for bad in ([0, 150, 120], [0, 100, 201], [5, 100, 200], [0, 190, 200]):
+        tcu = dev(np.asarray(bad, dtype=np.int32))
+        o = h3.varlen_attn_fwd_t(tq, tk, tv, tcu, 120 if bad == [0, 190, 200] else 150,
+                                 dev(pos), split, workspace=ws)
+        torch.cuda.synchronize()
+        assert h3.device_status_t(ws) == h3.H3_ERR_BAD_SEQLENS, bad
+    # a good call afterwards resets the status and works
+    o = h3.varlen_attn_fwd_t(tq, tk, tv, dev(cu), 100, dev(pos), split, workspace=ws)
+    torch.cuda.synchronize()
+    assert h3.device_status_t(ws) == h3.H3_OK
+    O, _ = oracle.attention_ref(q, k, v, cu, 0.125, pos, split)
+    assert_close_bf16(host_f64(o), O, "after bad calls")
+
+
+def test_empty_input_is_a_noop():
+    import torch
+    h3 = _h3()
+    z = torch.empty((0, 2, 64), dtype=torch.bfloat16, device="cuda")
+    cu = torch.zeros(2, dtype=torch.int32, device="cuda")
+    ws = h3.workspace_for(0, 2, 64, 1)
+    out = h3.varlen_attn_fwd_t(z, z, z, cu, 1, None, None, workspace=ws)
+    torch.cuda.synchronize()
+    assert out.shape == (0, 2, 64)
+    assert h3.device_status_t(ws) == h3.H3_OK
