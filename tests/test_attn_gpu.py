@@ -188,14 +188,25 @@ def test_uniform_scores_give_segment_mean():
 
 
 def test_skewed_keys_large_logits():
-    # keys offset by a large per-head constant: the running max moves a lot
+    # Keys offset by a large per-head constant: logits span ~11 units, the
+    # softmax is peaked and the running max moves by more than the lazy
+    # rescale threshold. With |k| ~ 6 the bf16 rounding of the rotated keys
+    # (the kernel rounds rotated q and k to bf16 before the MMA) alone moves
+    # the float64 answer by up to ~0.03, so the oracle is evaluated on q and k
+    # rotated in float64 and rounded to bf16 the same way (float64 -> float32
+    # -> bf16, round to nearest even).
     q, k, v, pos, cu, split = _case([1500], 2, 128, (32, 48, 48), seed=81)
     kk = oracle.bf16_bits_to_f64(k)
     kk[:, 0, :] += 3.0
     kk[700:, 1, :] += 6.0
     kb = synth.f32_to_bf16_bits(kk.astype(np.float32))
-    o, lse = _run(q, kb, v, cu, 1500, pos, split, 1.0 / math.sqrt(128))
-    O, L = oracle.attention_ref(q, kb, v, cu, 1.0 / math.sqrt(128), pos, split)
+    sc = 1.0 / math.sqrt(128)
+    o, lse = _run(q, kb, v, cu, 1500, pos, split, sc)
+    qr = oracle.rope_ref(oracle.bf16_bits_to_f64(q), pos, split, 1e4)
+    kr = oracle.rope_ref(oracle.bf16_bits_to_f64(kb), pos, split, 1e4)
+    qr = synth.f32_to_bf16_bits(qr.astype(np.float32))
+    kr = synth.f32_to_bf16_bits(kr.astype(np.float32))
+    O, L = oracle.attention_ref(qr, kr, v, cu, sc)
     assert_close_bf16(host_f64(o), O, "skewed")
     np.testing.assert_allclose(host_f64(lse), L, rtol=0, atol=2e-2)
 
