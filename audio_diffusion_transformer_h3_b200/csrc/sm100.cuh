@@ -223,6 +223,31 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// 2^x on the FMA and integer pipes instead of MUFU.
+// Method: Cody-Waite style range reduction x = j + f with j = rint(x)
+// (obtained by adding and subtracting 1.5 * 2^23, exact for |x| < 2^22) and
+// |f| <= 1/2; then 2^x = p(f) * 2^j, the 2^j applied by adding j to the
+// exponent field of p(f). p is a degree-3 polynomial fitted to 2^f on
+// [-1/2, 1/2] for minimum maximum relative error (iteratively reweighted
+// least squares): max relative error 7.6e-5, well below the 2^-9 relative
+// rounding of the bf16 P it feeds. x is clamped to >= -126 so the exponent
+// add cannot underflow (2^-126 is below anything that survives next to the
+// row maximum, which contributes 1).
+__device__ __forceinline__ float exp2_fma(float x) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    constexpr float c0 = 0.9999284744262695f, c1 = 0.6932608485221863f;
+    constexpr float c2 = 0.24260516464710236f, c3 = 0.05516925826668739f;
+    x = fmaxf(x, -126.0f);
+    const float t = __fadd_rn(x, kShift);     // kShift + rint(x)
+    const float r = __fadd_rn(t, -kShift);    // rint(x)
+    const float f = __fadd_rn(x, -r);         // x - rint(x), exact
+    float p = __fmaf_rn(c3, f, c2);
+    p = __fmaf_rn(p, f, c1);
+    p = __fmaf_rn(p, f, c0);
+    // low bits of t hold j: bits(t) * 2^23 == j << 23 modulo 2^32
+    return __uint_as_float(__float_as_uint(t) * 8388608u + __float_as_uint(p));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
