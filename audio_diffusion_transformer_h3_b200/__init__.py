@@ -6,7 +6,7 @@ the C names; the ``*_t`` helpers take torch tensors and call the same entry
 points with their pointers.
 
 The library is loaded from this directory (built in-tree by
-``python -m audio_diffusion_transformer_h3_b200.build`` or
+``python audio_diffusion_transformer_h3_b200/build.py`` or
 ``__graft_entry__.build()``). There is no fallback: if it is missing or does
 not load, importing this package raises.
 """
@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_HERE, "libh3attn.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"{LIB_PATH} is missing: build it with "
-        "`python -m audio_diffusion_transformer_h3_b200.build` (nvcc, sm_100a)")
+        "`python audio_diffusion_transformer_h3_b200/build.py` (nvcc, sm_100a)")
 _lib = ctypes.CDLL(LIB_PATH)
 
 # ----------------------------------------------------------------- C types
@@ -64,6 +64,10 @@ _lib.h3_varlen_attn_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _c.c_int32, _c.c_int
                                     h3_rope_cfg, _c.c_int64, _c.c_int32, _c.c_int32,
                                     _c.c_float, _P, _c.c_size_t, _P]
 _lib.h3_varlen_attn_fwd.restype = _c.c_int
+_lib.h3_varlen_attn_fwd_static.argtypes = [_P, _P, _P, _P, _P, _P, _c.c_int32, _c.c_int32, _P,
+                                           h3_rope_cfg, _c.c_int64, _c.c_int32, _c.c_int32,
+                                           _c.c_float, _P]
+_lib.h3_varlen_attn_fwd_static.restype = _c.c_int
 _lib.h3_read_device_status.argtypes = [_P, _P]
 _lib.h3_read_device_status.restype = _c.c_int
 _lib.h3_status_string.argtypes = [_c.c_int]
@@ -72,8 +76,12 @@ _lib.h3_last_cuda_error.argtypes = []
 _lib.h3_last_cuda_error.restype = _c.c_int32
 
 EXPORTED = ("h3_segment_tokens", "h3_build_positions", "h3_rope_apply", "h3_workspace_size",
-            "h3_varlen_attn_fwd", "h3_read_device_status", "h3_status_string",
-            "h3_last_cuda_error")
+            "h3_varlen_attn_fwd", "h3_varlen_attn_fwd_static", "h3_read_device_status",
+            "h3_status_string", "h3_last_cuda_error")
+
+# Scratch bytes compiled into the library for h3_varlen_attn_fwd_static
+# (H3_STATIC_WORKSPACE_BYTES in include/h3attn.h).
+H3_STATIC_WORKSPACE_BYTES = 256 + (64 << 20)
 
 
 class H3Error(RuntimeError):
@@ -124,6 +132,16 @@ def h3_varlen_attn_fwd(q: int, k: int, v: int, o: int, lse: int, cu_seqlens: int
     return int(_lib.h3_varlen_attn_fwd(q, k, v, o, lse, cu_seqlens, nseg, max_seqlen, pos, rope,
                                        N, H, D, softmax_scale, workspace, workspace_bytes,
                                        stream))
+
+
+def h3_varlen_attn_fwd_static(q: int, k: int, v: int, o: int, lse: int, cu_seqlens: int,
+                              nseg: int, max_seqlen: int, pos: int, rope: h3_rope_cfg, N: int,
+                              H: int, D: int, softmax_scale: float, stream: int) -> int:
+    """h3_varlen_attn_fwd without a caller workspace: for hosts that cannot
+    allocate device memory, the library's own compiled-in scratch is used
+    (N*H*D <= 2^25; calls on one device must not overlap on the GPU)."""
+    return int(_lib.h3_varlen_attn_fwd_static(q, k, v, o, lse, cu_seqlens, nseg, max_seqlen,
+                                              pos, rope, N, H, D, softmax_scale, stream))
 
 
 def h3_read_device_status(workspace: int, stream: int) -> int:

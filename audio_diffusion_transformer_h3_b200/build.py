@@ -1,6 +1,6 @@
 """Builds libh3attn.so in-tree with nvcc for sm_100a.
 
-    python -m audio_diffusion_transformer_h3_b200.build [--verbose]
+    python audio_diffusion_transformer_h3_b200/build.py [--verbose]
 
 The library is written next to this file so that it travels with the
 source tree; ``audio_diffusion_transformer_h3_b200`` loads it from there.
@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libh3attn.so")
 
-SOURCES = [os.path.join(CSRC, "h3attn.cu")]
+SOURCES = [os.path.join(CSRC, "h3attn.cu"), os.path.join(CSRC, "h3attn_static.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("sm100.cuh", "rope.cuh", "attn_fwd.cuh")] + [
     os.path.join(INCLUDE, "h3attn.h")]
 

@@ -146,6 +146,37 @@ h3_status h3_varlen_attn_fwd(const void *q, const void *k, const void *v, void *
                              int32_t D, float softmax_scale, void *workspace,
                              size_t workspace_bytes, h3_stream_t stream);
 
+/* Bytes of the scratch array compiled into the library for
+ * h3_varlen_attn_fwd_static: a 256-byte status block plus room for the
+ * rotated keys of N*H*D <= 2^25 elements (64 MiB of bf16). */
+#define H3_STATIC_WORKSPACE_BYTES (256u + (64u << 20))
+
+/* h3_varlen_attn_fwd for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is a deployment convenience. Hosts
+ * that own all device memory (their own arena or a fixed budget, allocation
+ * only at start-up) cannot give h3_varlen_attn_fwd a workspace; this call
+ * allocates nothing and uses a scratch array compiled into the library
+ * instead (H3_STATIC_WORKSPACE_BYTES of device memory on every device where
+ * it is used, held until the process exits). Arguments and results are those
+ * of h3_varlen_attn_fwd without the workspace pair.
+ *   Limit: N*H*D*2 + 256 <= H3_STATIC_WORKSPACE_BYTES (N*H*D <= 2^25), else
+ *          H3_ERR_WORKSPACE before anything is enqueued.
+ *   Set-up: the first call on a device looks up the array's device address
+ *          (cudaGetSymbolAddress, with that device current); make that first
+ *          call before any stream capture.
+ *   Sharing: every call on a device uses the same array. Calls that can run
+ *          concurrently on the GPU (different streams, no ordering) race on
+ *          it and must be serialised by the caller. Each call resets the
+ *          status word and rewrites all of the scratch it reads.
+ *   Device status: the array's status word is not exposed; a caller that
+ *          needs H3_ERR_BAD_SEQLENS / H3_ERR_DEVICE_TIMEOUT from the device
+ *          uses h3_varlen_attn_fwd with its own workspace. */
+h3_status h3_varlen_attn_fwd_static(const void *q, const void *k, const void *v, void *o,
+                                    float *lse, const int32_t *cu_seqlens, int32_t nseg,
+                                    int32_t max_seqlen, const float *pos, h3_rope_cfg rope,
+                                    int64_t N, int32_t H, int32_t D, float softmax_scale,
+                                    h3_stream_t stream);
+
 /* Waits for `stream`, then returns the device status word of the last call
  * that used `workspace` (H3_OK, H3_ERR_BAD_SEQLENS or H3_ERR_DEVICE_TIMEOUT),
  * or H3_ERR_CUDA if the copy fails. */
