@@ -10,7 +10,8 @@
 //
 // One CTA computes two 128-row query tiles (Q0, Q1) of one (segment, head)
 // against every 128-row key/value tile of the segment:
-//   warp 9      TMA producer: Q0/Q1 once, then K_j and V_j through a
+//   warp 9      TMA producer (converged warp, elected lane issues): Q0/Q1
+//               once, then K_j and V_j through a
 //               two-stage ring (128B-swizzled boxes of 128 rows x 64 cols);
 //   warps 0-7   softmax, one thread per query row (warpgroup t owns Q_t and
 //               TMEM lanes 0..127): rotate their Q row in shared memory
@@ -20,7 +21,8 @@
 //               O rescale skipped unless the max grows by more than 2^8),
 //               write P_t as bf16 into the same TMEM columns, and finally
 //               normalise O_t and store bf16 rows (and the LSE);
-//   warp 8      MMA issuer (one thread): S_t = Q_t K_j^T (A, B from shared
+//   warp 8      MMA issuer (the whole warp runs the schedule, one elected
+//               lane issues): S_t = Q_t K_j^T (A, B from shared
 //               memory) and O_t += P_t V_j (A = P from TMEM, B = V from
 //               shared memory), ordered PV0(j-1), S0(j), PV1(j-1), S1(j) so
 //               the tensor core works on one tile while the other tile's
@@ -157,99 +159,113 @@ __global__ void __launch_bounds__(320, 1)
 
     if (warp == 9) {
         // ============================ TMA producer ============================
-        if (lane == 0) {
-            mbar_arrive_expect_tx(&bars[B_QFULL], 2 * C::TILE_BYTES);
-            for (int t = 0; t < 2; ++t)
-                for (int b = 0; b < C::NBOX; ++b)
+        // Converged warp; the elected lane issues the copies and expect_tx.
+        const uint32_t leader = elect_one();
+        if (leader) mbar_arrive_expect_tx(&bars[B_QFULL], 2 * C::TILE_BYTES);
+        for (int t = 0; t < 2; ++t)
+            for (int b = 0; b < C::NBOX; ++b)
+                if (leader)
                     tma_load_3d(smem + C::OFF_Q + t * C::TILE_BYTES + b * C::BOX_BYTES, &tmQ,
                                 &bars[B_QFULL], b * 64, head, q0 + t * C::BM);
-            int last_k = -1, last_v = -1;
-            for (int j = 0; j < n_kv; ++j) {
-                const int s = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
-                const int kv0 = seg_start + j * C::BN;
-                if (!mbar_wait(&bars[B_KEMPTY + s], ph ^ 1, abort)) { raise_abort(abort, p.status); break; }
+        int last_k = -1, last_v = -1;
+        for (int j = 0; j < n_kv; ++j) {
+            const int s = j & 1;
+            const uint32_t ph = (j >> 1) & 1;
+            const int kv0 = seg_start + j * C::BN;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_KEMPTY + s], ph ^ 1, abort))) {
+                if (leader) raise_abort(abort, p.status);
+                break;
+            }
+            if (leader) {
                 mbar_arrive_expect_tx(&bars[B_KFULL + s], C::TILE_BYTES);
                 for (int b = 0; b < C::NBOX; ++b)
                     tma_load_3d(smem + C::OFF_K + s * C::TILE_BYTES + b * C::BOX_BYTES, &tmK,
                                 &bars[B_KFULL + s], b * 64, head, kv0);
-                last_k = j;
-                if (!mbar_wait(&bars[B_VEMPTY + s], ph ^ 1, abort)) { raise_abort(abort, p.status); break; }
+            }
+            last_k = j;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_VEMPTY + s], ph ^ 1, abort))) {
+                if (leader) raise_abort(abort, p.status);
+                break;
+            }
+            if (leader) {
                 mbar_arrive_expect_tx(&bars[B_VFULL + s], C::TILE_BYTES);
                 for (int b = 0; b < C::NBOX; ++b)
                     tma_load_3d(smem + C::OFF_V + s * C::TILE_BYTES + b * C::BOX_BYTES, &tmV,
                                 &bars[B_VFULL + s], b * 64, head, kv0);
-                last_v = j;
             }
-            if (*abort) {
-                // let the copies still in flight land before shared memory is released
-                mbar_wait(&bars[B_QFULL], 0, nullptr);
-                for (int j = (last_k > 0 ? last_k - 1 : 0); j <= last_k; ++j)
-                    mbar_wait(&bars[B_KFULL + (j & 1)], (j >> 1) & 1, nullptr);
-                for (int j = (last_v > 0 ? last_v - 1 : 0); j <= last_v; ++j)
-                    mbar_wait(&bars[B_VFULL + (j & 1)], (j >> 1) & 1, nullptr);
-            }
+            last_v = j;
+        }
+        if (*abort) {
+            // let the copies still in flight land before shared memory is released
+            mbar_wait(&bars[B_QFULL], 0, nullptr);
+            for (int j = (last_k > 0 ? last_k - 1 : 0); j <= last_k; ++j)
+                mbar_wait(&bars[B_KFULL + (j & 1)], (j >> 1) & 1, nullptr);
+            for (int j = (last_v > 0 ? last_v - 1 : 0); j <= last_v; ++j)
+                mbar_wait(&bars[B_VFULL + (j & 1)], (j >> 1) & 1, nullptr);
         }
         __syncwarp();
     } else if (warp == 8) {
         // ============================ MMA issuer ==============================
-        if (lane == 0) {
-            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
-            const uint32_t sQ = smem_u32(smem + C::OFF_Q);
-            const uint32_t sK = smem_u32(smem + C::OFF_K);
-            const uint32_t sV = smem_u32(smem + C::OFF_V);
-            bool ok = mbar_wait(&bars[B_QREADY], 0, abort);
-            tc_fence_after();
-            for (int j = 0; ok && j <= n_kv; ++j) {
-                for (int t = 0; ok && t < 2; ++t) {
-                    const uint32_t colS = t ? C::COL_S1 : C::COL_S0;
-                    const uint32_t colO = t ? C::COL_O1 : C::COL_O0;
-                    if (j > 0) {  // O_t += P_t(j-1) V_{j-1}
-                        const int jj = j - 1;
-                        const int vs = jj & 1;
-                        ok = mbar_wait(&bars[B_PFULL + t], jj & 1, abort);
-                        if (ok && t == 0) ok = mbar_wait(&bars[B_VFULL + vs], (jj >> 1) & 1, abort);
+        // The whole warp runs this schedule (waits included) so that it stays
+        // converged; only the elected lane issues the MMAs and commits.
+        const uint32_t leader = elect_one();
+        constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
+        const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+        const uint32_t sK = smem_u32(smem + C::OFF_K);
+        const uint32_t sV = smem_u32(smem + C::OFF_V);
+        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_QREADY], 0, abort));
+        tc_fence_after();
+        for (int j = 0; ok && j <= n_kv; ++j) {
+            for (int t = 0; ok && t < 2; ++t) {
+                const uint32_t colS = t ? C::COL_S1 : C::COL_S0;
+                const uint32_t colO = t ? C::COL_O1 : C::COL_O0;
+                if (j > 0) {  // O_t += P_t(j-1) V_{j-1}
+                    const int jj = j - 1;
+                    const int vs = jj & 1;
+                    bool w = mbar_wait(&bars[B_PFULL + t], jj & 1, abort);
+                    if (w && t == 0) w = mbar_wait(&bars[B_VFULL + vs], (jj >> 1) & 1, abort);
+                    ok = __all_sync(0xffffffffu, w);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t vbase = sV + vs * C::TILE_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < C::BN / 16; ++kk) {
+                        // V tile [128 keys][D] is MN-major for B: 8 key rows at 128 B,
+                        // groups of 8 rows at SBO = 1024 B, 64-col boxes at LBO.
+                        const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::BOX_BYTES, 1024);
+                        umma_ts_w(tmem + colO, tmem + colS + kk * 8, bdesc, IDESC_O,
+                                  (jj > 0 || kk > 0) ? 1u : 0u, leader);
+                    }
+                    if (j == n_kv) umma_commit_w(&bars[B_OFULL + t], leader);
+                    if (t == 1) umma_commit_w(&bars[B_VEMPTY + vs], leader);
+                }
+                if (j < n_kv) {  // S_t = Q_t K_j^T
+                    const int ks = j & 1;
+                    if (t == 0) {
+                        ok = __all_sync(0xffffffffu,
+                                        mbar_wait(&bars[B_KFULL + ks], (j >> 1) & 1, abort));
                         if (!ok) break;
                         tc_fence_after();
-                        const uint32_t vbase = sV + vs * C::TILE_BYTES;
-#pragma unroll
-                        for (int kk = 0; kk < C::BN / 16; ++kk) {
-                            // V tile [128 keys][D] is MN-major for B: 8 key rows at 128 B,
-                            // groups of 8 rows at SBO = 1024 B, 64-col boxes at LBO.
-                            const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::BOX_BYTES, 1024);
-                            umma_ts(tmem + colO, tmem + colS + kk * 8, bdesc, IDESC_O,
-                                    (jj > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        if (j == n_kv) umma_commit(&bars[B_OFULL + t]);
-                        if (t == 1) umma_commit(&bars[B_VEMPTY + vs]);
                     }
-                    if (j < n_kv) {  // S_t = Q_t K_j^T
-                        const int ks = j & 1;
-                        if (t == 0) {
-                            ok = mbar_wait(&bars[B_KFULL + ks], (j >> 1) & 1, abort);
-                            if (!ok) break;
-                            tc_fence_after();
-                        }
-                        const uint32_t qbase = sQ + t * C::TILE_BYTES;
-                        const uint32_t kbase = sK + ks * C::TILE_BYTES;
+                    const uint32_t qbase = sQ + t * C::TILE_BYTES;
+                    const uint32_t kbase = sK + ks * C::TILE_BYTES;
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-                            const uint64_t adesc = sdesc_sw128(qbase + off, 16, 1024);
-                            const uint64_t bdesc = sdesc_sw128(kbase + off, 16, 1024);
-                            umma_ss(tmem + colS, adesc, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit(&bars[B_SFULL + t]);
-                        if (t == 1) umma_commit(&bars[B_KEMPTY + ks]);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+                        const uint64_t adesc = sdesc_sw128(qbase + off, 16, 1024);
+                        const uint64_t bdesc = sdesc_sw128(kbase + off, 16, 1024);
+                        umma_ss_w(tmem + colS, adesc, bdesc, IDESC_S, kk > 0 ? 1u : 0u, leader);
                     }
+                    umma_commit_w(&bars[B_SFULL + t], leader);
+                    if (t == 1) umma_commit_w(&bars[B_KEMPTY + ks], leader);
                 }
             }
-            if (!ok) {
-                raise_abort(abort, p.status);
-                umma_commit(&bars[B_DRAIN]);  // completes once every issued MMA is done
-                mbar_wait(&bars[B_DRAIN], 0, nullptr);
-            }
+        }
+        if (!ok) {
+            if (leader) raise_abort(abort, p.status);
+            umma_commit_w(&bars[B_DRAIN], leader);  // completes once every issued MMA is done
+            mbar_wait(&bars[B_DRAIN], 0, nullptr);
         }
         __syncwarp();
     } else {
