@@ -41,6 +41,15 @@
 #include "rope.cuh"
 #include "sm100.cuh"
 
+// Column pairs out of every eight whose exponentials run on the FMA pipe
+// (exp2_fma) instead of MUFU, and whether the row max uses 3-input max.
+#ifndef H3_FMA_EXP2_PAIRS
+#define H3_FMA_EXP2_PAIRS 0
+#endif
+#ifndef H3_MAX3
+#define H3_MAX3 0
+#endif
+
 namespace h3 {
 
 enum : int { kStatusOk = 0, kStatusTimeout = 6, kStatusBadSeqlens = 7 };
@@ -136,7 +145,7 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(&bars[B_VFULL + s], 1);
             mbar_init(&bars[B_VEMPTY + s], 1);
             mbar_init(&bars[B_SFULL + s], 1);
-            mbar_init(&bars[B_PFULL + s], 128);
+            mbar_init(&bars[B_PFULL + s], 4);
             mbar_init(&bars[B_OFULL + s], 1);
         }
         mbar_init(&bars[B_DRAIN], 1);
@@ -323,9 +332,22 @@ __global__ void __launch_bounds__(320, 1)
                 for (int c = 0; c < 128; ++c)
                     if (c >= kv_valid) s[c] = __float_as_uint(-INFINITY);
             }
-            float mx = __uint_as_float(s[0]);
+            // row max over 128 keys in 8 independent chains (ALU throughput, not latency)
+            float mq[8];
 #pragma unroll
-            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+            for (int i = 0; i < 8; ++i) mq[i] = __uint_as_float(s[i]);
+#if H3_MAX3
+#pragma unroll
+            for (int c = 8; c < 128; c += 16)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    mq[i] = fmax3(mq[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 8 + i]));
+#else
+#pragma unroll
+            for (int c = 8; c < 128; ++c) mq[c & 7] = fmaxf(mq[c & 7], __uint_as_float(s[c]));
+#endif
+            const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
+                                   fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
             const float m_new = mx * sl2;
             bool need = false;
             if (j == 0) {
@@ -339,6 +361,7 @@ __global__ void __launch_bounds__(320, 1)
                 m_used = m_new;
             }
             const float nm = -m_used;
+            float lq[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             uint32_t pk[64];
             if (kv_valid < C::BN) {
                 // keys past the segment end get P = 0 exactly (also when the
@@ -349,18 +372,29 @@ __global__ void __launch_bounds__(320, 1)
                         ? ex2_approx(fmaf(__uint_as_float(s[2 * c]), sl2, nm)) : 0.0f;
                     const float p1 = (2 * c + 1 < kv_valid)
                         ? ex2_approx(fmaf(__uint_as_float(s[2 * c + 1]), sl2, nm)) : 0.0f;
-                    l += p0 + p1;
+                    lq[c & 3] += p0 + p1;
                     pk[c] = pack_bf16x2(p0, p1);
                 }
             } else {
+                // H3_FMA_EXP2_PAIRS column pairs of every eight on the FMA pipe
+                // (exp2_fma), the rest on MUFU (ex2.approx)
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * c]), sl2, nm));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * c + 1]), sl2, nm));
-                    l += p0 + p1;
+                    const float x0 = fmaf(__uint_as_float(s[2 * c]), sl2, nm);
+                    const float x1 = fmaf(__uint_as_float(s[2 * c + 1]), sl2, nm);
+                    float p0, p1;
+                    if ((c & 7) >= 8 - H3_FMA_EXP2_PAIRS) {
+                        p0 = exp2_fma(x0);
+                        p1 = exp2_fma(x1);
+                    } else {
+                        p0 = ex2_approx(x0);
+                        p1 = ex2_approx(x1);
+                    }
+                    lq[c & 3] += p0 + p1;
                     pk[c] = pack_bf16x2(p0, p1);
                 }
             }
+            l += (lq[0] + lq[1]) + (lq[2] + lq[3]);
             if (__any_sync(0xffffffffu, need)) {
                 // O_t holds P V up to tile j-1 (S_t(j) completing implies every
                 // earlier MMA completed); rescale it before P_t(j) is released.
@@ -378,7 +412,8 @@ __global__ void __launch_bounds__(320, 1)
             tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars[B_PFULL + t]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[B_PFULL + t]);  // one arrival per warp
         }
 
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_OFULL + t], 0, abort));

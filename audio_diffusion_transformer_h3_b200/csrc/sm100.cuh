@@ -271,6 +271,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// max(a, b, c) in one instruction (sm_100 three-input form).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // 2^x on the FMA and integer pipes instead of MUFU.
 // Method: Cody-Waite style range reduction x = j + f with j = rint(x)
 // (obtained by adding and subtracting 1.5 * 2^23, exact for |x| < 2^22) and
