@@ -68,6 +68,8 @@ _lib.h3_varlen_attn_fwd_static.argtypes = [_P, _P, _P, _P, _P, _P, _c.c_int32, _
                                            h3_rope_cfg, _c.c_int64, _c.c_int32, _c.c_int32,
                                            _c.c_float, _P]
 _lib.h3_varlen_attn_fwd_static.restype = _c.c_int
+_lib.h3_selftest_bounded_wait.argtypes = [_P, _c.c_size_t, _c.c_int64, _P]
+_lib.h3_selftest_bounded_wait.restype = _c.c_int
 _lib.h3_read_device_status.argtypes = [_P, _P]
 _lib.h3_read_device_status.restype = _c.c_int
 _lib.h3_status_string.argtypes = [_c.c_int]
@@ -76,8 +78,8 @@ _lib.h3_last_cuda_error.argtypes = []
 _lib.h3_last_cuda_error.restype = _c.c_int32
 
 EXPORTED = ("h3_segment_tokens", "h3_build_positions", "h3_rope_apply", "h3_workspace_size",
-            "h3_varlen_attn_fwd", "h3_varlen_attn_fwd_static", "h3_read_device_status",
-            "h3_status_string", "h3_last_cuda_error")
+            "h3_varlen_attn_fwd", "h3_varlen_attn_fwd_static", "h3_selftest_bounded_wait",
+            "h3_read_device_status", "h3_status_string", "h3_last_cuda_error")
 
 # Scratch bytes compiled into the library for h3_varlen_attn_fwd_static
 # (H3_STATIC_WORKSPACE_BYTES in include/h3attn.h).
@@ -142,6 +144,11 @@ def h3_varlen_attn_fwd_static(q: int, k: int, v: int, o: int, lse: int, cu_seqle
     (N*H*D <= 2^25; calls on one device must not overlap on the GPU)."""
     return int(_lib.h3_varlen_attn_fwd_static(q, k, v, o, lse, cu_seqlens, nseg, max_seqlen,
                                               pos, rope, N, H, D, softmax_scale, stream))
+
+
+def h3_selftest_bounded_wait(workspace: int, workspace_bytes: int, limit_cycles: int,
+                             stream: int) -> int:
+    return int(_lib.h3_selftest_bounded_wait(workspace, workspace_bytes, limit_cycles, stream))
 
 
 def h3_read_device_status(workspace: int, stream: int) -> int:

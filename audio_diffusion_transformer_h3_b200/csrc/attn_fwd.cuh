@@ -96,6 +96,22 @@ __device__ __forceinline__ void raise_abort(volatile int *abort, int *status) {
     atomicCAS(status, kStatusOk, kStatusTimeout);
 }
 
+// Self-test of the bounded wait: one warp waits on an mbarrier that nothing
+// arrives on, with a cycle limit, exactly as the attention kernel's waits do;
+// when the wait gives up it records H3_ERR_DEVICE_TIMEOUT in the status word
+// and the kernel returns normally.
+__global__ void __launch_bounds__(32, 1) bounded_wait_selftest_kernel(int *status,
+                                                                       long long limit_cycles) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar, 0, nullptr, limit_cycles));
+    if (!ok && threadIdx.x == 0) atomicCAS(status, kStatusOk, kStatusTimeout);
+}
+
 template <int D>
 __global__ void __launch_bounds__(320, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ,

@@ -312,6 +312,23 @@ h3_status h3_varlen_attn_fwd(const void *q, const void *k, const void *v, void *
     return e == cudaSuccess ? H3_OK : cuda_fail(e);
 }
 
+h3_status h3_selftest_bounded_wait(void *workspace, size_t workspace_bytes,
+                                   int64_t limit_cycles, h3_stream_t stream) {
+    if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < kStatusBytes)
+        return H3_ERR_WORKSPACE;
+    if (limit_cycles < 1 || limit_cycles > 4000000000LL) return H3_ERR_INVALID_ARG;
+    DeviceInfo *d = nullptr;
+    h3_status st = device_info(&d);
+    if (st != H3_OK) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    int *status = static_cast<int *>(workspace);
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), cs);
+    if (e != cudaSuccess) return cuda_fail(e);
+    h3::bounded_wait_selftest_kernel<<<1, 32, 0, cs>>>(status, static_cast<long long>(limit_cycles));
+    e = cudaGetLastError();
+    return e == cudaSuccess ? H3_OK : cuda_fail(e);
+}
+
 h3_status h3_read_device_status(const void *workspace, h3_stream_t stream) {
     if (workspace == nullptr) return H3_ERR_WORKSPACE;
     int host = 0;

@@ -59,13 +59,14 @@ constexpr long long kWaitLimitCycles = 2000000000LL;
 // *abort (a CTA-wide flag in shared memory) becomes non-zero when abort is
 // not null. Never traps.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          const volatile int *abort) {
+                                          const volatile int *abort,
+                                          long long limit_cycles = kWaitLimitCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (abort != nullptr && *abort != 0) return false;
-        if (clock64() - t0 > kWaitLimitCycles) return false;
+        if (clock64() - t0 > limit_cycles) return false;
     }
 }
 

@@ -61,16 +61,24 @@ def measured_peaks() -> dict:
 
 
 def recorded_traffic(workload: str):
-    """DRAM bytes per attention launch from the committed ncu summary, or None
-    if the summary is missing or was taken on a different kernel source."""
-    p = os.path.join(PROFILE_DIR, f"attn_fwd_{workload}_traffic.json")
+    """DRAM bytes per attention launch from the committed ncu summary
+    ``profiles/attn_fwd_<workload>_traffic.txt`` (``key: value`` lines), or
+    None if it is missing or was taken on a different kernel source."""
+    p = os.path.join(PROFILE_DIR, f"attn_fwd_{workload}_traffic.txt")
     if not os.path.exists(p):
         return None
+    rec = {}
     with open(p) as f:
-        d = json.load(f)
-    if d.get("kernel_source_hash") != kernel_source_hash():
+        for line in f:
+            if ":" in line and not line.lstrip().startswith("#"):
+                k, v = line.split(":", 1)
+                rec[k.strip()] = v.strip()
+    if rec.get("kernel_source_hash") != kernel_source_hash():
         return None
-    return d.get("dram_bytes_per_launch")
+    try:
+        return int(rec["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 class ClockSampler:

@@ -177,6 +177,16 @@ h3_status h3_varlen_attn_fwd_static(const void *q, const void *k, const void *v,
                                     int64_t N, int32_t H, int32_t D, float softmax_scale,
                                     h3_stream_t stream);
 
+/* Failure-detection self-test (no counterpart on the pages): one warp runs the
+ * same bounded mbarrier wait the attention kernel uses, on a barrier that
+ * nothing arrives on, giving up after `limit_cycles` SM clock cycles
+ * (1 .. 4e9; the attention kernel's own limit is 2e9, about one second). The
+ * kernel then writes H3_ERR_DEVICE_TIMEOUT to the status word of `workspace`
+ * (>= 256 bytes, 256-byte aligned) and returns normally, so the CUDA context
+ * stays usable; read it with h3_read_device_status. Asynchronous on `stream`. */
+h3_status h3_selftest_bounded_wait(void *workspace, size_t workspace_bytes,
+                                   int64_t limit_cycles, h3_stream_t stream);
+
 /* Waits for `stream`, then returns the device status word of the last call
  * that used `workspace` (H3_OK, H3_ERR_BAD_SEQLENS or H3_ERR_DEVICE_TIMEOUT),
  * or H3_ERR_CUDA if the copy fails. */

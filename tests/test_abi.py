@@ -126,3 +126,10 @@ def test_host_positions_errors():
     arr = (h3.h3_segment_layout * 1)(seg)
     assert h3._lib.h3_build_positions(arr, 1, buf.ctypes.data, 4, None) == h3.H3_ERR_INVALID_ARG
     assert h3.h3_segment_tokens(h3.h3_segment_layout(-1, 0, 0, 0, 0, 0, 0, 0, 0, 0)) == -1
+
+
+def test_selftest_host_argument_errors():
+    assert h3.h3_selftest_bounded_wait(0, 256, 1000, 0) == h3.H3_ERR_WORKSPACE
+    assert h3.h3_selftest_bounded_wait(0x10010, 256, 1000, 0) == h3.H3_ERR_WORKSPACE
+    assert h3.h3_selftest_bounded_wait(0x10000, 128, 1000, 0) == h3.H3_ERR_WORKSPACE
+    assert h3.h3_selftest_bounded_wait(0x10000, 256, 0, 0) == h3.H3_ERR_INVALID_ARG

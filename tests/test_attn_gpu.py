@@ -243,3 +243,20 @@ def test_empty_input_is_a_noop():
     torch.cuda.synchronize()
     assert out.shape == (0, 2, 64)
     assert h3.device_status_t(ws) == h3.H3_OK
+
+
+def test_bounded_wait_gives_up_and_reports_timeout():
+    # a wait on a barrier that nothing arrives on ends after its cycle limit
+    # with H3_ERR_DEVICE_TIMEOUT in the status word; the context stays usable
+    import torch
+    h3 = _h3()
+    ws = h3.workspace_for(0, 1, 64, 1)
+    stream = torch.cuda.current_stream().cuda_stream
+    st = h3.h3_selftest_bounded_wait(ws.data_ptr(), ws.numel(), 2_000_000, stream)
+    assert st == h3.H3_OK
+    assert h3.device_status_t(ws) == h3.H3_ERR_DEVICE_TIMEOUT
+    # the next call on the same context works and resets the status
+    q, k, v, pos, cu, split = _case([100, 60], 2, 64, (16, 24, 24), seed=101)
+    o = _run(q, k, v, cu, 100, pos, split, 0.125, return_lse=False)
+    O, _ = oracle.attention_ref(q, k, v, cu, 0.125, pos, split)
+    assert_close_bf16(host_f64(o), O, "after timeout self-test")
