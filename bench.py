@@ -142,6 +142,30 @@ def workload_config(wl) -> dict:
             "L2 flushed (256 MB write) before every timed step"}
 
 
+# ---------------------------------------------------------- multi-rank helpers
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Seed of rank ``rank``'s own packed workload (weak scaling: every rank
+    draws an independent batch of the same shape)."""
+    return base_seed + 7919 * rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Maximum of ``x`` over all ranks (the timed region is the slowest rank's)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_rank_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank's FLOPs over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- CPU oracle
 
 def cpu_oracle_sample(wl, q, k, v, pos, cu, budget_s: float):
@@ -215,7 +239,7 @@ def run_ours(args, wl, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    seed = wl.the_seed + 7919 * rank
+    seed = rank_seed(wl.the_seed, rank)
     q, k, v = synth.draw_qkv(wl, seed=seed)
     pos, cu = h3.h3_build_positions(wl.segments)
     N, H, D = wl.n_tokens, wl.heads, wl.head_dim
@@ -250,13 +274,6 @@ def run_ours(args, wl, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -278,10 +295,10 @@ def run_ours(args, wl, rank, world, local_rank):
         torch.cuda.synchronize()
     barrier()
     step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]))
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), world, dev)
     if h3.device_status_t(ws) != h3.H3_OK:
         raise RuntimeError("device status not ok after timed region")
-    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_tflops(world, flops_step, args.steps, total_ms)
     mean_step_ms = float(np.mean(step_ms))
 
     # ---- end-to-end through the public API with host buffers ----
@@ -308,8 +325,8 @@ def run_ours(args, wl, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = world * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = job_tflops(world, flops_step, args.steps, e2e_ms)
 
     peaks = measured_peaks()
     achieved = flops_step / (mean_step_ms * 1e-3) / 1e12

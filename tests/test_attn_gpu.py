@@ -260,3 +260,36 @@ def test_bounded_wait_gives_up_and_reports_timeout():
     o = _run(q, k, v, cu, 100, pos, split, 0.125, return_lse=False)
     O, _ = oracle.attention_ref(q, k, v, cu, 0.125, pos, split)
     assert_close_bf16(host_f64(o), O, "after timeout self-test")
+
+
+def test_head_subset_equals_full_call_bitwise():
+    # heads are independent units: the kernel on a head group (what each rank
+    # of the Ulysses wrapper runs) reproduces those heads of the full call
+    q, k, v, pos, cu, split = _case([300, 129, 700], 8, 128, (32, 48, 48), seed=111)
+    o_full = host_bits(_run(q, k, v, cu, 700, pos, split, 0.09, return_lse=False))
+    for h0, h1 in ((0, 4), (4, 8), (2, 3)):
+        sub = [np.ascontiguousarray(x[:, h0:h1]) for x in (q, k, v)]
+        o = host_bits(_run(*sub, cu, 700, pos, split, 0.09, return_lse=False))
+        assert np.array_equal(o, o_full[:, h0:h1])
+
+
+def test_ulysses_single_rank_is_the_kernel():
+    import os
+    import torch
+    import torch.distributed as dist
+    from audio_diffusion_transformer_h3_b200.ulysses import ulysses_attention
+    h3 = _h3()
+    if not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29561")
+        dist.init_process_group("nccl", rank=0, world_size=1)
+    try:
+        q, k, v, pos, cu, split = _case([200, 333], 4, 128, (32, 48, 48), seed=121)
+        tq, tk, tv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+        tcu, tpos = dev(cu), dev(pos)
+        a = ulysses_attention(tq, tk, tv, tcu, 333, tpos, split, 1e4, 0.1)
+        b = h3.varlen_attn_fwd_t(tq, tk, tv, tcu, 333, tpos, split, 1e4, 0.1)
+        torch.cuda.synchronize()
+        assert np.array_equal(host_bits(a), host_bits(b))
+    finally:
+        dist.destroy_process_group()
