@@ -68,6 +68,12 @@ _lib.h3_varlen_attn_fwd_static.argtypes = [_P, _P, _P, _P, _P, _P, _c.c_int32, _
                                            h3_rope_cfg, _c.c_int64, _c.c_int32, _c.c_int32,
                                            _c.c_float, _P]
 _lib.h3_varlen_attn_fwd_static.restype = _c.c_int
+_lib.h3_varlen_attn_fwd_skip.argtypes = [_P, _P, _P, _P, _P, _P, _c.c_int32, _c.c_int32, _P,
+                                         h3_rope_cfg, _c.c_int64, _c.c_int32, _c.c_int32,
+                                         _c.c_float, _c.c_float, _P, _c.c_size_t, _P]
+_lib.h3_varlen_attn_fwd_skip.restype = _c.c_int
+_lib.h3_read_skip_count.argtypes = [_P, _P, _c.POINTER(_c.c_uint64)]
+_lib.h3_read_skip_count.restype = _c.c_int
 _lib.h3_selftest_bounded_wait.argtypes = [_P, _c.c_size_t, _c.c_int64, _P]
 _lib.h3_selftest_bounded_wait.restype = _c.c_int
 _lib.h3_read_device_status.argtypes = [_P, _P]
@@ -78,7 +84,8 @@ _lib.h3_last_cuda_error.argtypes = []
 _lib.h3_last_cuda_error.restype = _c.c_int32
 
 EXPORTED = ("h3_segment_tokens", "h3_build_positions", "h3_rope_apply", "h3_workspace_size",
-            "h3_varlen_attn_fwd", "h3_varlen_attn_fwd_static", "h3_selftest_bounded_wait",
+            "h3_varlen_attn_fwd", "h3_varlen_attn_fwd_skip", "h3_read_skip_count",
+            "h3_varlen_attn_fwd_static", "h3_selftest_bounded_wait",
             "h3_read_device_status", "h3_status_string", "h3_last_cuda_error")
 
 # Scratch bytes compiled into the library for h3_varlen_attn_fwd_static
@@ -134,6 +141,21 @@ def h3_varlen_attn_fwd(q: int, k: int, v: int, o: int, lse: int, cu_seqlens: int
     return int(_lib.h3_varlen_attn_fwd(q, k, v, o, lse, cu_seqlens, nseg, max_seqlen, pos, rope,
                                        N, H, D, softmax_scale, workspace, workspace_bytes,
                                        stream))
+
+
+def h3_varlen_attn_fwd_skip(q: int, k: int, v: int, o: int, lse: int, cu_seqlens: int,
+                            nseg: int, max_seqlen: int, pos: int, rope: h3_rope_cfg, N: int,
+                            H: int, D: int, softmax_scale: float, skip_threshold: float,
+                            workspace: int, workspace_bytes: int, stream: int) -> int:
+    return int(_lib.h3_varlen_attn_fwd_skip(q, k, v, o, lse, cu_seqlens, nseg, max_seqlen, pos,
+                                            rope, N, H, D, softmax_scale, skip_threshold,
+                                            workspace, workspace_bytes, stream))
+
+
+def h3_read_skip_count(workspace: int, stream: int) -> int:
+    n = ctypes.c_uint64(0)
+    _check(_lib.h3_read_skip_count(workspace, stream, ctypes.byref(n)), "h3_read_skip_count")
+    return int(n.value)
 
 
 def h3_varlen_attn_fwd_static(q: int, k: int, v: int, o: int, lse: int, cu_seqlens: int,
@@ -241,6 +263,38 @@ def varlen_attn_fwd_t(q, k, v, cu_seqlens, max_seqlen: int, pos=None, split=None
                             workspace.data_ptr(), workspace.numel(), _stream(stream))
     _check(st, "h3_varlen_attn_fwd")
     return (out, lse) if return_lse else out
+
+
+def varlen_attn_fwd_skip_t(q, k, v, cu_seqlens, max_seqlen: int, skip_threshold: float,
+                           pos=None, split=None, theta: float = 10000.0,
+                           softmax_scale: Optional[float] = None, out=None,
+                           return_lse: bool = False, workspace=None, stream=None):
+    """Skip-softmax variant through h3_varlen_attn_fwd_skip; the number of
+    skipped (32-row block, key tile) pairs is read with skip_count_t(workspace)."""
+    import torch
+    _thd(q, "q"); _thd(k, "k"); _thd(v, "v")
+    N, H, D = q.shape
+    nseg = int(cu_seqlens.numel()) - 1
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((H, N), dtype=torch.float32, device=q.device) if return_lse else None
+    if workspace is None:
+        workspace = workspace_for(N, H, D, nseg, q.device)
+    scale = (1.0 / math.sqrt(D)) if softmax_scale is None else float(softmax_scale)
+    rope = rope_cfg(split, theta) if pos is not None else h3_rope_cfg(0, 0, 0, 0.0)
+    st = h3_varlen_attn_fwd_skip(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr() if lse is not None else 0,
+                                 cu_seqlens.data_ptr(), nseg, int(max_seqlen),
+                                 pos.data_ptr() if pos is not None else 0, rope, N, H, D, scale,
+                                 float(skip_threshold), workspace.data_ptr(), workspace.numel(),
+                                 _stream(stream))
+    _check(st, "h3_varlen_attn_fwd_skip")
+    return (out, lse) if return_lse else out
+
+
+def skip_count_t(workspace, stream=None) -> int:
+    """Skipped (32-row block, key tile) pairs of the last skip call on ``workspace`` (syncs)."""
+    return h3_read_skip_count(workspace.data_ptr(), _stream(stream))
 
 
 def device_status_t(workspace, stream=None) -> int:

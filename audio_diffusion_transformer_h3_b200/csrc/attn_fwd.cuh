@@ -62,6 +62,8 @@ struct AttnParams {
     int *status;                // device status word
     int32_t nseg, max_seqlen, N, H;
     float scale_log2;           // softmax_scale * log2(e)
+    float skip_log2;            // log2(skip threshold) (skip-softmax variant only)
+    unsigned long long *skip_count;  // skipped (32-row block, key tile) pairs, or nullptr
     RopeTable rope;
 };
 
@@ -112,7 +114,14 @@ __global__ void __launch_bounds__(32, 1) bounded_wait_selftest_kernel(int *statu
     if (!ok && threadIdx.x == 0) atomicCAS(status, kStatusOk, kStatusTimeout);
 }
 
-template <int D>
+// SKIP: skip-softmax variant ("MiniMax H3" vLLM-Omni recipe, section
+// "Attention Backends", Skip-Softmax). For a 32-row block (one softmax warp)
+// and a key tile j > 0, if every row of the block has
+// exp(tile max - running max) < threshold (rows past the segment end do not
+// vote), the block stores P = 0 without computing exponentials and leaves its
+// running state unchanged; if all four blocks of a query tile skip, the MMA
+// warp also drops that tile's PV.
+template <int D, bool SKIP>
 __global__ void __launch_bounds__(320, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK,
@@ -151,6 +160,8 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + B_COUNT);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    // skip-softmax: per query tile and softmax warp, 1 + the last key tile it skipped
+    volatile uint32_t *skipword = reinterpret_cast<volatile uint32_t *>(tmem_slot + 2);
 
     if (tid == 0) {
         mbar_init(&bars[B_QFULL], 1);
@@ -166,6 +177,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         mbar_init(&bars[B_DRAIN], 1);
         *abort = 0;
+        for (int i = 0; i < 8; ++i) skipword[i] = 0;
         fence_mbar_init();
     }
     if (warp == 8) {
@@ -254,8 +266,15 @@ __global__ void __launch_bounds__(320, 1)
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t vbase = sV + vs * C::TILE_BYTES;
+                    bool skip_pv = false;
+                    if constexpr (SKIP) {
+                        const uint32_t tag = static_cast<uint32_t>(jj + 1);
+                        skip_pv = skipword[t * 4 + 0] == tag && skipword[t * 4 + 1] == tag &&
+                                  skipword[t * 4 + 2] == tag && skipword[t * 4 + 3] == tag;
+                    }
 #pragma unroll
                     for (int kk = 0; kk < C::BN / 16; ++kk) {
+                        if (skip_pv) break;
                         // V tile [128 keys][D] is MN-major for B: 8 key rows at 128 B,
                         // groups of 8 rows at SBO = 1024 B, 64-col boxes at LBO.
                         const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::BOX_BYTES, 1024);
@@ -331,6 +350,7 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive(&bars[B_QREADY]);
 
         float m_used = -INFINITY, l = 0.f;
+        float m_run = -INFINITY;  // true running row max (skip-softmax decision)
         const float sl2 = p.scale_log2;
         for (int j = 0; ok && j < n_kv; ++j) {
             ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + t], j & 1, abort));
@@ -365,6 +385,33 @@ __global__ void __launch_bounds__(320, 1)
             const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
                                    fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
             const float m_new = mx * sl2;
+            if constexpr (SKIP) {
+                if (j == 0) {
+                    m_run = m_new;
+                } else {
+                    // rows past the segment end do not vote
+                    const bool negligible = qrow >= seg_end || m_new - m_run < p.skip_log2;
+                    if (__all_sync(0xffffffffu, negligible)) {
+                        uint32_t z[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) z[i] = 0u;
+                        tmem_st32(tS + 0, z);
+                        tmem_st32(tS + 32, z);
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            skipword[t * 4 + (warp & 3)] = static_cast<uint32_t>(j + 1);
+                            // blocks with no row inside the segment are not counted
+                            if (p.skip_count != nullptr && q0 + t * C::BM + (warp & 3) * 32 < seg_end)
+                                atomicAdd(p.skip_count, 1ull);
+                            mbar_arrive(&bars[B_PFULL + t]);
+                        }
+                        continue;
+                    }
+                    m_run = fmaxf(m_run, m_new);
+                }
+            }
             bool need = false;
             if (j == 0) {
                 m_used = m_new;

@@ -81,10 +81,16 @@ h3_status device_info(DeviceInfo **out) {
             return cuda_fail(e);
         d.sm100 = (major == 10 && minor == 0);
         if (d.sm100) {
-            if ((e = cudaFuncSetAttribute(h3::attn_fwd_kernel<128>,
+            if ((e = cudaFuncSetAttribute(h3::attn_fwd_kernel<128, false>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           h3::AttnCfg<128>::SMEM_BYTES)) != cudaSuccess ||
-                (e = cudaFuncSetAttribute(h3::attn_fwd_kernel<64>,
+                (e = cudaFuncSetAttribute(h3::attn_fwd_kernel<64, false>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          h3::AttnCfg<64>::SMEM_BYTES)) != cudaSuccess ||
+                (e = cudaFuncSetAttribute(h3::attn_fwd_kernel<128, true>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          h3::AttnCfg<128>::SMEM_BYTES)) != cudaSuccess ||
+                (e = cudaFuncSetAttribute(h3::attn_fwd_kernel<64, true>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           h3::AttnCfg<64>::SMEM_BYTES)) != cudaSuccess)
                 return cuda_fail(e);
@@ -148,6 +154,91 @@ h3_status launch_rope(const void *x, void *out, const float *pos, int64_t N, int
         h3::rope_apply_kernel<64><<<grid, 256, 0, st>>>(
             static_cast<const uint4 *>(x), static_cast<uint4 *>(out), pos, N, H, rt);
     cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? H3_OK : cuda_fail(e);
+}
+
+h3_status attn_call(const void *q, const void *k, const void *v, void *o, float *lse,
+                    const int32_t *cu_seqlens, int32_t nseg, int32_t max_seqlen,
+                    const float *pos, h3_rope_cfg rope, int64_t N, int32_t H, int32_t D,
+                    float softmax_scale, void *workspace, size_t workspace_bytes,
+                    h3_stream_t stream, bool skip, float skip_threshold) {
+    if (N < 0 || N > INT32_MAX - 1 || H < 1 || H > 65535 || nseg < 1 || nseg > 65535)
+        return H3_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return H3_ERR_UNSUPPORTED;
+    if (!std::isfinite(softmax_scale) || softmax_scale < 0.0f) return H3_ERR_INVALID_ARG;
+    if (cu_seqlens == nullptr) return H3_ERR_INVALID_ARG;
+    if (N > 0 && (q == nullptr || k == nullptr || v == nullptr || o == nullptr))
+        return H3_ERR_INVALID_ARG;
+    if (N > 0 && (max_seqlen < 1 || max_seqlen > N)) return H3_ERR_INVALID_ARG;
+    h3::RopeTable rt;
+    std::memset(&rt, 0, sizeof(rt));
+    if (pos != nullptr && !make_rope_table(rope, D, &rt)) return H3_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(pos, 4) || !aligned(lse, 4) || !aligned(cu_seqlens, 4))
+        return H3_ERR_MISALIGNED;
+    if (workspace == nullptr || !aligned(workspace, 256) ||
+        workspace_bytes < h3_workspace_size(N, H, D, nseg))
+        return H3_ERR_WORKSPACE;
+
+    DeviceInfo *d = nullptr;
+    h3_status st = device_info(&d);
+    if (st != H3_OK) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    int *status = static_cast<int *>(workspace);
+    // status word (and, for the skip variant, the skipped-block counter at byte 8)
+    cudaError_t e = cudaMemsetAsync(status, 0, skip ? 16 : sizeof(int), cs);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (N == 0) return H3_OK;
+
+    // keys rotated once into the workspace (the same rotation the attention
+    // kernel applies to each query tile)
+    const void *k_src = k;
+    if (pos != nullptr) {
+        void *k_rot = static_cast<uint8_t *>(workspace) + kStatusBytes;
+        st = launch_rope(k, k_rot, pos, N, H, D, rt, d->sms, cs);
+        if (st != H3_OK) return st;
+        k_src = k_rot;
+    }
+
+    CUtensorMap tq, tk, tv;
+    if ((st = make_thd_map(&tq, q, N, H, D)) != H3_OK) return st;
+    if ((st = make_thd_map(&tk, k_src, N, H, D)) != H3_OK) return st;
+    if ((st = make_thd_map(&tv, v, N, H, D)) != H3_OK) return st;
+
+    h3::AttnParams p;
+    p.cu_seqlens = cu_seqlens;
+    p.pos = pos;
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    p.status = status;
+    p.nseg = nseg;
+    p.max_seqlen = max_seqlen;
+    p.N = static_cast<int32_t>(N);
+    p.H = H;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.skip_log2 = skip ? static_cast<float>(std::log2(static_cast<double>(skip_threshold))) : 0.0f;
+    p.skip_count = skip ? reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + 8)
+                        : nullptr;
+    p.rope = rt;
+
+    const dim3 grid(static_cast<unsigned>((max_seqlen + 255) / 256), static_cast<unsigned>(H),
+                    static_cast<unsigned>(nseg));
+    if (D == 128) {
+        if (skip)
+            h3::attn_fwd_kernel<128, true><<<grid, h3::AttnCfg<128>::THREADS,
+                                             h3::AttnCfg<128>::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+        else
+            h3::attn_fwd_kernel<128, false><<<grid, h3::AttnCfg<128>::THREADS,
+                                              h3::AttnCfg<128>::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+    } else {
+        if (skip)
+            h3::attn_fwd_kernel<64, true><<<grid, h3::AttnCfg<64>::THREADS,
+                                            h3::AttnCfg<64>::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+        else
+            h3::attn_fwd_kernel<64, false><<<grid, h3::AttnCfg<64>::THREADS,
+                                             h3::AttnCfg<64>::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+    }
+    e = cudaGetLastError();
     return e == cudaSuccess ? H3_OK : cuda_fail(e);
 }
 
@@ -245,71 +336,32 @@ h3_status h3_varlen_attn_fwd(const void *q, const void *k, const void *v, void *
                              const float *pos, h3_rope_cfg rope, int64_t N, int32_t H,
                              int32_t D, float softmax_scale, void *workspace,
                              size_t workspace_bytes, h3_stream_t stream) {
-    if (N < 0 || N > INT32_MAX - 1 || H < 1 || H > 65535 || nseg < 1 || nseg > 65535)
-        return H3_ERR_INVALID_ARG;
-    if (D != 64 && D != 128) return H3_ERR_UNSUPPORTED;
-    if (!std::isfinite(softmax_scale) || softmax_scale < 0.0f) return H3_ERR_INVALID_ARG;
-    if (cu_seqlens == nullptr) return H3_ERR_INVALID_ARG;
-    if (N > 0 && (q == nullptr || k == nullptr || v == nullptr || o == nullptr))
-        return H3_ERR_INVALID_ARG;
-    if (N > 0 && (max_seqlen < 1 || max_seqlen > N)) return H3_ERR_INVALID_ARG;
-    h3::RopeTable rt;
-    std::memset(&rt, 0, sizeof(rt));
-    if (pos != nullptr && !make_rope_table(rope, D, &rt)) return H3_ERR_INVALID_ARG;
-    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
-        !aligned(pos, 4) || !aligned(lse, 4) || !aligned(cu_seqlens, 4))
-        return H3_ERR_MISALIGNED;
-    if (workspace == nullptr || !aligned(workspace, 256) ||
-        workspace_bytes < h3_workspace_size(N, H, D, nseg))
-        return H3_ERR_WORKSPACE;
+    return attn_call(q, k, v, o, lse, cu_seqlens, nseg, max_seqlen, pos, rope, N, H, D,
+                     softmax_scale, workspace, workspace_bytes, stream, false, 0.0f);
+}
 
-    DeviceInfo *d = nullptr;
-    h3_status st = device_info(&d);
-    if (st != H3_OK) return st;
+h3_status h3_varlen_attn_fwd_skip(const void *q, const void *k, const void *v, void *o,
+                                  float *lse, const int32_t *cu_seqlens, int32_t nseg,
+                                  int32_t max_seqlen, const float *pos, h3_rope_cfg rope,
+                                  int64_t N, int32_t H, int32_t D, float softmax_scale,
+                                  float skip_threshold, void *workspace, size_t workspace_bytes,
+                                  h3_stream_t stream) {
+    if (!(skip_threshold >= 0.0f && skip_threshold <= 1.0f)) return H3_ERR_INVALID_ARG;
+    return attn_call(q, k, v, o, lse, cu_seqlens, nseg, max_seqlen, pos, rope, N, H, D,
+                     softmax_scale, workspace, workspace_bytes, stream, true, skip_threshold);
+}
+
+h3_status h3_read_skip_count(const void *workspace, h3_stream_t stream, uint64_t *count) {
+    if (workspace == nullptr) return H3_ERR_WORKSPACE;
+    if (count == nullptr) return H3_ERR_INVALID_ARG;
+    unsigned long long host = 0;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    int *status = static_cast<int *>(workspace);
-    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), cs);
+    cudaError_t e = cudaMemcpyAsync(&host, static_cast<const uint8_t *>(workspace) + 8,
+                                    sizeof(host), cudaMemcpyDeviceToHost, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
     if (e != cudaSuccess) return cuda_fail(e);
-    if (N == 0) return H3_OK;
-
-    // keys rotated once into the workspace (the same rotation the attention
-    // kernel applies to each query tile)
-    const void *k_src = k;
-    if (pos != nullptr) {
-        void *k_rot = static_cast<uint8_t *>(workspace) + kStatusBytes;
-        st = launch_rope(k, k_rot, pos, N, H, D, rt, d->sms, cs);
-        if (st != H3_OK) return st;
-        k_src = k_rot;
-    }
-
-    CUtensorMap tq, tk, tv;
-    if ((st = make_thd_map(&tq, q, N, H, D)) != H3_OK) return st;
-    if ((st = make_thd_map(&tk, k_src, N, H, D)) != H3_OK) return st;
-    if ((st = make_thd_map(&tv, v, N, H, D)) != H3_OK) return st;
-
-    h3::AttnParams p;
-    p.cu_seqlens = cu_seqlens;
-    p.pos = pos;
-    p.o = static_cast<__nv_bfloat16 *>(o);
-    p.lse = lse;
-    p.status = status;
-    p.nseg = nseg;
-    p.max_seqlen = max_seqlen;
-    p.N = static_cast<int32_t>(N);
-    p.H = H;
-    p.scale_log2 = softmax_scale * 1.4426950408889634f;
-    p.rope = rt;
-
-    const dim3 grid(static_cast<unsigned>((max_seqlen + 255) / 256), static_cast<unsigned>(H),
-                    static_cast<unsigned>(nseg));
-    if (D == 128)
-        h3::attn_fwd_kernel<128><<<grid, h3::AttnCfg<128>::THREADS,
-                                   h3::AttnCfg<128>::SMEM_BYTES, cs>>>(tq, tk, tv, p);
-    else
-        h3::attn_fwd_kernel<64><<<grid, h3::AttnCfg<64>::THREADS,
-                                  h3::AttnCfg<64>::SMEM_BYTES, cs>>>(tq, tk, tv, p);
-    e = cudaGetLastError();
-    return e == cudaSuccess ? H3_OK : cuda_fail(e);
+    *count = static_cast<uint64_t>(host);
+    return H3_OK;
 }
 
 h3_status h3_selftest_bounded_wait(void *workspace, size_t workspace_bytes,

@@ -364,6 +364,65 @@ def run_ours(args, wl, rank, world, local_rank):
     return 0
 
 
+def run_skip(args, wl, rank, world, local_rank):
+    """Skip-softmax variant on inputs with frame-group locality (one group per
+    1008-token frame, synth.draw_group_case): dense-equivalent TFLOP/s (the
+    dense FLOPs over the time of the skip call), the skipped share of
+    (32-row block, key tile) pairs, and the dense kernel's time on the same
+    inputs for comparison. Single process only."""
+    import torch
+
+    import audio_diffusion_transformer_h3_b200 as h3
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    q, k, v, cu = synth.draw_group_case(wl.seg_lens, wl.heads, wl.head_dim, group_len=1008,
+                                        amp=15.0, eps=0.05, seed=rank_seed(wl.the_seed, rank))
+    pos, _ = h3.h3_build_positions(wl.segments)
+    N, H, D = wl.n_tokens, wl.heads, wl.head_dim
+
+    def bf(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    dq, dk, dv, dcu = bf(q), bf(k), bf(v), torch.from_numpy(cu).to(dev)
+    do = torch.empty_like(dq)
+    ws = h3.workspace_for(N, H, D, len(wl.seg_lens), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    # no RoPE here: the group codes are the locality structure
+    ms_skip = timed(lambda: h3.varlen_attn_fwd_skip_t(dq, dk, dv, dcu, wl.max_seqlen,
+                                                      args.skip_threshold, None, None, wl.theta,
+                                                      wl.softmax_scale, out=do, workspace=ws,
+                                                      stream=stream))
+    skipped = h3.skip_count_t(ws)
+    ms_dense = timed(lambda: h3.varlen_attn_fwd_t(dq, dk, dv, dcu, wl.max_seqlen, None, None,
+                                                  wl.theta, wl.softmax_scale, out=do,
+                                                  workspace=ws, stream=stream))
+    pairs = sum(((L + 31) // 32) * ((L + 127) // 128 - 1) for L in wl.seg_lens) * H
+    line = {"metric": "skip-softmax fused varlen joint attention fwd, dense-equivalent TFLOP/s",
+            "value": wl.flops() / (ms_skip * 1e-3) / 1e12, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_skip,
+            "higher_is_better": True, "dtype": "bf16",
+            "data": "synthetic frame-group locality (synth.draw_group_case, 1008-token groups)",
+            "config": workload_config(wl), "skip_threshold": args.skip_threshold,
+            "skipped_fraction": skipped / pairs, "dense_ms_same_inputs": ms_dense,
+            "speedup_vs_dense": ms_dense / ms_skip, "gpu_launches": args.steps}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -374,6 +433,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-threshold", type=float, default=None,
+                    help="time the skip-softmax variant on frame-group inputs instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -385,6 +446,8 @@ def main():
 
     if args.impl == "reference":
         return run_reference(args, wl, rank, world)
+    if args.skip_threshold is not None:
+        return run_skip(args, wl, rank, world, local_rank)
 
     if world > 1:
         import datetime

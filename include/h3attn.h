@@ -146,6 +146,33 @@ h3_status h3_varlen_attn_fwd(const void *q, const void *k, const void *v, void *
                              int32_t D, float softmax_scale, void *workspace,
                              size_t workspace_bytes, h3_stream_t stream);
 
+/* Skip-Softmax variant of h3_varlen_attn_fwd (lossy). "MiniMax H3" vLLM-Omni
+ * recipe, section "Attention Backends": Skip-Softmax sparse attention skips
+ * tiles whose softmax contribution is below a direct threshold (0.05 in the
+ * pages' example; which denoising steps stay dense is the caller's choice).
+ * Reading used here: keys are taken in tiles of 128 from the segment start,
+ * query rows in blocks of 32 inside 128-row tiles from the segment start. A
+ * block skips key tile j > 0 when, for every row of the block,
+ * exp(tile's max score - row's running max score) < skip_threshold (scores
+ * include softmax_scale; skipped tiles never raise the running max). The
+ * result is softmax attention over the keys of the kept tiles.
+ *   skip_threshold: 0 <= t <= 1 (0 never skips), else H3_ERR_INVALID_ARG.
+ *   workspace: as for h3_varlen_attn_fwd; bytes [8, 16) receive the number of
+ *              skipped (32-row block, key tile) pairs (h3_read_skip_count).
+ * All other arguments, results and errors are those of h3_varlen_attn_fwd. */
+h3_status h3_varlen_attn_fwd_skip(const void *q, const void *k, const void *v, void *o,
+                                  float *lse, const int32_t *cu_seqlens, int32_t nseg,
+                                  int32_t max_seqlen, const float *pos, h3_rope_cfg rope,
+                                  int64_t N, int32_t H, int32_t D, float softmax_scale,
+                                  float skip_threshold, void *workspace, size_t workspace_bytes,
+                                  h3_stream_t stream);
+
+/* Waits for `stream`, then writes to *count the number of (32-row block, key
+ * tile) pairs the last h3_varlen_attn_fwd_skip call on `workspace` skipped.
+ * H3_ERR_WORKSPACE / H3_ERR_INVALID_ARG on null pointers, H3_ERR_CUDA if the
+ * copy fails. */
+h3_status h3_read_skip_count(const void *workspace, h3_stream_t stream, uint64_t *count);
+
 /* Bytes of the scratch array compiled into the library for
  * h3_varlen_attn_fwd_static: a 256-byte status block plus room for the
  * rotated keys of N*H*D <= 2^25 elements (64 MiB of bf16). */

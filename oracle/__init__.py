@@ -19,6 +19,8 @@ What it computes, and the passages it follows:
 * ``attention``   -- non-causal softmax attention inside each packed
   segment ("MiniMax H3" vLLM-Omni recipe, section "Step execution and
   continuous batching": one attention document per packed request).
+* ``skip_softmax`` -- the lossy Skip-Softmax variant that drops negligible
+  key tiles ("MiniMax H3" vLLM-Omni recipe, section "Attention Backends").
 
 Readings where the pages say nothing (pair layout, frequency schedule,
 audio-token clock, reference layout) are listed in the design notes of the
@@ -38,3 +40,4 @@ from .attention import (  # noqa: F401
     attention_dense_bruteforce,
     attention_rows_ref,
 )
+from .skip_softmax import attention_skip_ref, attention_skip_rows_ref  # noqa: F401

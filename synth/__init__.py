@@ -15,6 +15,7 @@ from .configs import (  # noqa: F401
     workload,
     draw_qkv,
     draw_random_case,
+    draw_group_case,
     f32_to_bf16_bits,
     cu_seqlens_of,
 )

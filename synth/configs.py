@@ -203,3 +203,31 @@ def draw_random_case(seg_lens: Sequence[int], heads: int, head_dim: int, seed: i
     v = f32_to_bf16_bits(rng.standard_normal((N, heads, head_dim), dtype=np.float32))
     pos = (rng.random((N, 3), dtype=np.float32) * np.float32(pos_range)).astype(np.float32)
     return q, k, v, pos, cu_seqlens_of(seg_lens)
+
+
+def draw_group_case(seg_lens: Sequence[int], heads: int, head_dim: int, group_len: int,
+                    amp: float, eps: float, seed: int):
+    """Inputs with frame-group locality for the skip-softmax variant.
+
+    Token i of a segment belongs to group g = i // group_len (counted from the
+    segment start); its q and k are amp * e_(g mod head_dim) plus eps * N(0,1)
+    noise per channel, v is N(0,1). Same-group scores are ~amp^2 and all others
+    ~0, so a key tile either matters to a query or is clearly negligible.
+    Recipe: default_rng(seed), noise for q, then k, then v, float32, rounded to
+    bf16 (RNE). Returns q, k, v bits and cu_seqlens.
+    """
+    N = int(sum(seg_lens))
+    rng = np.random.default_rng(seed)
+    code = np.zeros((N, head_dim), dtype=np.float32)
+    start = 0
+    for L in seg_lens:
+        g = (np.arange(L) // group_len) % head_dim
+        code[start + np.arange(L), g] = np.float32(amp)
+        start += L
+    out = []
+    for _ in range(2):
+        x = rng.standard_normal((N, heads, head_dim), dtype=np.float32) * np.float32(eps)
+        x += code[:, None, :]
+        out.append(f32_to_bf16_bits(x))
+    v = f32_to_bf16_bits(rng.standard_normal((N, heads, head_dim), dtype=np.float32))
+    return out[0], out[1], v, cu_seqlens_of(seg_lens)
