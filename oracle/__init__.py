@@ -21,6 +21,9 @@ What it computes, and the passages it follows:
   continuous batching": one attention document per packed request).
 * ``skip_softmax`` -- the lossy Skip-Softmax variant that drops negligible
   key tiles ("MiniMax H3" vLLM-Omni recipe, section "Attention Backends").
+* ``qkv_rope``    -- the qkv projection with RoPE applied to q and k in its
+  epilogue ("MiniMax-H3 Reference" Space README, section "AoTI-compiled
+  blocks": rotary epilogues around the block's matmuls).
 
 Readings where the pages say nothing (pair layout, frequency schedule,
 audio-token clock, reference layout) are listed in the design notes of the
@@ -41,3 +44,4 @@ from .attention import (  # noqa: F401
     attention_rows_ref,
 )
 from .skip_softmax import attention_skip_ref, attention_skip_rows_ref  # noqa: F401
+from .qkv_rope import qkv_rope_ref  # noqa: F401
