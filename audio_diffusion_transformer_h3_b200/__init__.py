@@ -72,6 +72,9 @@ _lib.h3_varlen_attn_fwd_skip.argtypes = [_P, _P, _P, _P, _P, _P, _c.c_int32, _c.
                                          h3_rope_cfg, _c.c_int64, _c.c_int32, _c.c_int32,
                                          _c.c_float, _c.c_float, _P, _c.c_size_t, _P]
 _lib.h3_varlen_attn_fwd_skip.restype = _c.c_int
+_lib.h3_qkv_rope_gemm.argtypes = [_P, _P, _P, _P, _P, _P, h3_rope_cfg, _c.c_int64, _c.c_int32,
+                                  _c.c_int32, _c.c_int32, _P, _c.c_size_t, _P]
+_lib.h3_qkv_rope_gemm.restype = _c.c_int
 _lib.h3_read_skip_count.argtypes = [_P, _P, _c.POINTER(_c.c_uint64)]
 _lib.h3_read_skip_count.restype = _c.c_int
 _lib.h3_selftest_bounded_wait.argtypes = [_P, _c.c_size_t, _c.c_int64, _P]
@@ -85,6 +88,7 @@ _lib.h3_last_cuda_error.restype = _c.c_int32
 
 EXPORTED = ("h3_segment_tokens", "h3_build_positions", "h3_rope_apply", "h3_workspace_size",
             "h3_varlen_attn_fwd", "h3_varlen_attn_fwd_skip", "h3_read_skip_count",
+            "h3_qkv_rope_gemm",
             "h3_varlen_attn_fwd_static", "h3_selftest_bounded_wait",
             "h3_read_device_status", "h3_status_string", "h3_last_cuda_error")
 
@@ -150,6 +154,13 @@ def h3_varlen_attn_fwd_skip(q: int, k: int, v: int, o: int, lse: int, cu_seqlens
     return int(_lib.h3_varlen_attn_fwd_skip(q, k, v, o, lse, cu_seqlens, nseg, max_seqlen, pos,
                                             rope, N, H, D, softmax_scale, skip_threshold,
                                             workspace, workspace_bytes, stream))
+
+
+def h3_qkv_rope_gemm(x: int, w: int, q: int, k: int, v: int, pos: int, rope: h3_rope_cfg,
+                     N: int, K: int, H: int, D: int, workspace: int, workspace_bytes: int,
+                     stream: int) -> int:
+    return int(_lib.h3_qkv_rope_gemm(x, w, q, k, v, pos, rope, N, K, H, D, workspace,
+                                     workspace_bytes, stream))
 
 
 def h3_read_skip_count(workspace: int, stream: int) -> int:
@@ -290,6 +301,31 @@ def varlen_attn_fwd_skip_t(q, k, v, cu_seqlens, max_seqlen: int, skip_threshold:
                                  _stream(stream))
     _check(st, "h3_varlen_attn_fwd_skip")
     return (out, lse) if return_lse else out
+
+
+def qkv_rope_gemm_t(x, w, heads: int, head_dim: int, pos=None, split=None,
+                    theta: float = 10000.0, out=None, workspace=None, stream=None):
+    """(q, k, v) [N, H, D] bf16 through h3_qkv_rope_gemm: the projection
+    x [N, K] @ w[3*H*D, K]^T with RoPE applied to q and k in its epilogue."""
+    import torch
+    for t, name in ((x, "x"), (w, "w")):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 2 and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA bfloat16 matrix")
+    N, K = x.shape
+    if tuple(w.shape) != (3 * heads * head_dim, K):
+        raise ValueError(f"w must be [3*H*D, K] = [{3 * heads * head_dim}, {K}]")
+    if out is None:
+        out = tuple(torch.empty((N, heads, head_dim), dtype=torch.bfloat16, device=x.device)
+                    for _ in range(3))
+    q, k, v = out
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=x.device)
+    rope = rope_cfg(split, theta) if pos is not None else h3_rope_cfg(0, 0, 0, 0.0)
+    st = h3_qkv_rope_gemm(x.data_ptr(), w.data_ptr(), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                          pos.data_ptr() if pos is not None else 0, rope, N, K, heads,
+                          head_dim, workspace.data_ptr(), workspace.numel(), _stream(stream))
+    _check(st, "h3_qkv_rope_gemm")
+    return q, k, v
 
 
 def skip_count_t(workspace, stream=None) -> int:

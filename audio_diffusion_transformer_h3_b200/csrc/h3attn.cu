@@ -3,7 +3,7 @@
 // Host side only: argument validation, the rotary frequency table, TMA
 // descriptors, launches on the caller's stream, and the host position
 // builder. Every step of the device path runs in the kernels of
-// rope.cuh and attn_fwd.cuh; nothing here computes on the host except
+// rope.cuh, attn_fwd.cuh and qkv_gemm.cuh; nothing here computes on the host except
 // positions (which the pages place on the host: "MiniMax H3 on Moore Threads
 // MUSA", section "MUSA validation").
 #include <cuda.h>
@@ -16,6 +16,7 @@
 
 #include "h3attn.h"
 #include "attn_fwd.cuh"
+#include "qkv_gemm.cuh"
 #include "rope.cuh"
 
 namespace {
@@ -28,6 +29,9 @@ h3_status cuda_fail(cudaError_t e) {
 }
 
 constexpr size_t kStatusBytes = 256;
+
+// Row tiles of the QKV GEMM that sweep the column tiles together (L2 reuse).
+constexpr int32_t kQkvGroupM = 32;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -92,7 +96,13 @@ h3_status device_info(DeviceInfo **out) {
                                           h3::AttnCfg<128>::SMEM_BYTES)) != cudaSuccess ||
                 (e = cudaFuncSetAttribute(h3::attn_fwd_kernel<64, true>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          h3::AttnCfg<64>::SMEM_BYTES)) != cudaSuccess)
+                                          h3::AttnCfg<64>::SMEM_BYTES)) != cudaSuccess ||
+                (e = cudaFuncSetAttribute(h3::qkv_rope_gemm_kernel<128>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          h3::QkvCfg::SMEM_BYTES)) != cudaSuccess ||
+                (e = cudaFuncSetAttribute(h3::qkv_rope_gemm_kernel<64>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          h3::QkvCfg::SMEM_BYTES)) != cudaSuccess)
                 return cuda_fail(e);
         }
         d.ready = true;
@@ -135,6 +145,24 @@ h3_status make_thd_map(CUtensorMap *map, const void *base, int64_t N, int H, int
     const cuuint32_t box[3] = {64, 1, 128};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    return H3_OK;
+}
+
+// TMA map over a row-major bf16 [rows, cols] matrix: dims (cols, rows), box
+// (64, box_rows), 128-byte swizzle, zero fill out of bounds.
+h3_status make_2d_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols,
+                      uint32_t box_rows) {
+    EncodeTiledFn enc = encode_tiled();
+    if (enc == nullptr) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -349,6 +377,64 @@ h3_status h3_varlen_attn_fwd_skip(const void *q, const void *k, const void *v, v
     if (!(skip_threshold >= 0.0f && skip_threshold <= 1.0f)) return H3_ERR_INVALID_ARG;
     return attn_call(q, k, v, o, lse, cu_seqlens, nseg, max_seqlen, pos, rope, N, H, D,
                      softmax_scale, workspace, workspace_bytes, stream, true, skip_threshold);
+}
+
+h3_status h3_qkv_rope_gemm(const void *x, const void *w, void *q, void *k, void *v,
+                           const float *pos, h3_rope_cfg rope, int64_t N, int32_t K,
+                           int32_t H, int32_t D, void *workspace, size_t workspace_bytes,
+                           h3_stream_t stream) {
+    if (N < 0 || N > INT32_MAX - 256 || H < 1 || K < 64 || K > (1 << 20) || (K % 64) != 0)
+        return H3_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return H3_ERR_UNSUPPORTED;
+    const int64_t HD = static_cast<int64_t>(H) * D;
+    if ((HD % 256) != 0 || 3 * HD > (1 << 20)) return H3_ERR_INVALID_ARG;
+    if (N > 0 && (x == nullptr || w == nullptr || q == nullptr || k == nullptr || v == nullptr))
+        return H3_ERR_INVALID_ARG;
+    h3::RopeTable rt;
+    std::memset(&rt, 0, sizeof(rt));
+    if (pos != nullptr && !make_rope_table(rope, D, &rt)) return H3_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w, 16) || !aligned(q, 16) || !aligned(k, 16) ||
+        !aligned(v, 16) || !aligned(pos, 4))
+        return H3_ERR_MISALIGNED;
+    if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < kStatusBytes)
+        return H3_ERR_WORKSPACE;
+    DeviceInfo *d = nullptr;
+    h3_status st = device_info(&d);
+    if (st != H3_OK) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    int *status = static_cast<int *>(workspace);
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), cs);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (N == 0) return H3_OK;
+
+    using C = h3::QkvCfg;
+    h3::QkvParams p;
+    p.q = static_cast<__nv_bfloat16 *>(q);
+    p.k = static_cast<__nv_bfloat16 *>(k);
+    p.v = static_cast<__nv_bfloat16 *>(v);
+    p.pos = pos;
+    p.status = status;
+    p.N = static_cast<int32_t>(N);
+    p.K = K;
+    p.HD = static_cast<int32_t>(HD);
+    p.n_row_tiles = static_cast<int32_t>((N + C::BM - 1) / C::BM);
+    p.n_col_tiles = static_cast<int32_t>(3 * HD / C::BN);
+    const int64_t n_tiles = static_cast<int64_t>(p.n_row_tiles) * p.n_col_tiles;
+    if (n_tiles > INT32_MAX) return H3_ERR_INVALID_ARG;
+    p.n_tiles = static_cast<int32_t>(n_tiles);
+    p.group_m = kQkvGroupM;
+    p.rope = rt;
+
+    CUtensorMap tx, tw;
+    if ((st = make_2d_map(&tx, x, N, K, C::BM)) != H3_OK) return st;
+    if ((st = make_2d_map(&tw, w, 3 * HD, K, C::BN)) != H3_OK) return st;
+    const int grid = static_cast<int>(n_tiles < d->sms ? n_tiles : d->sms);
+    if (D == 128)
+        h3::qkv_rope_gemm_kernel<128><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tx, tw, p);
+    else
+        h3::qkv_rope_gemm_kernel<64><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tx, tw, p);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? H3_OK : cuda_fail(e);
 }
 
 h3_status h3_read_skip_count(const void *workspace, h3_stream_t stream, uint64_t *count) {

@@ -173,6 +173,35 @@ h3_status h3_varlen_attn_fwd_skip(const void *q, const void *k, const void *v, v
  * copy fails. */
 h3_status h3_read_skip_count(const void *workspace, h3_stream_t stream, uint64_t *count);
 
+/* QKV projection with the rotary embedding fused into its epilogue: the step
+ * that produces this path's q, k, v inside a DiT block. "MiniMax-H3
+ * Reference" Space README, section "AoTI-compiled blocks" (rotary epilogues
+ * around the block's matmuls); "MiniMax H3" vLLM-Omni recipe, section "Online
+ * FP8 quantization" (the attention's qkv projection is one of the DiT
+ * linears; BF16 here). Computes, with HD = H*D,
+ *     Y = x w^T                                   (fp32 accumulation)
+ *     q = RoPE(Y[:, 0:HD]),  k = RoPE(Y[:, HD:2HD]),  v = Y[:, 2HD:3HD]
+ * with RoPE as in h3_rope_apply (same table, pair layout and rounding
+ * sequence) but applied to the fp32 accumulator, each output rounded once to
+ * bf16 (round to nearest even). With pos NULL no rotation is applied and
+ * `rope` is ignored.
+ *   x        : device bf16 [N, K] row-major, 16-byte aligned.
+ *   w        : device bf16 [3*H*D, K] row-major (the linear layer's weight:
+ *              rows [0, HD) make q, [HD, 2HD) k, [2HD, 3HD) v), 16-byte aligned.
+ *   q, k, v  : device bf16 [N, H, D] each, 16-byte aligned, overlapping
+ *              neither each other nor x, w.
+ *   pos      : device fp32 [N, 3] or NULL.
+ *   N >= 0 (N = 0 is a no-op), N < 2^31; K a multiple of 64, 64 <= K <= 2^20;
+ *   D in {64, 128}; H >= 1 with H*D a multiple of 256 and 3*H*D <= 2^20.
+ *   workspace: device, 256-byte aligned, >= 256 bytes (its status word, which
+ *              a timed-out bounded wait sets to H3_ERR_DEVICE_TIMEOUT; read
+ *              it with h3_read_device_status). Reset by every call.
+ * One persistent kernel launch (one CTA per SM), deterministic. */
+h3_status h3_qkv_rope_gemm(const void *x, const void *w, void *q, void *k, void *v,
+                           const float *pos, h3_rope_cfg rope, int64_t N, int32_t K,
+                           int32_t H, int32_t D, void *workspace, size_t workspace_bytes,
+                           h3_stream_t stream);
+
 /* Bytes of the scratch array compiled into the library for
  * h3_varlen_attn_fwd_static: a 256-byte status block plus room for the
  * rotated keys of N*H*D <= 2^25 elements (64 MiB of bf16). */

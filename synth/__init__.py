@@ -18,4 +18,7 @@ from .configs import (  # noqa: F401
     draw_group_case,
     f32_to_bf16_bits,
     cu_seqlens_of,
+    QkvProjection,
+    QKV_PROJECTION,
+    draw_linear_case,
 )

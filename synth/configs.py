@@ -231,3 +231,39 @@ def draw_group_case(seg_lens: Sequence[int], heads: int, head_dim: int, group_le
         out.append(f32_to_bf16_bits(x))
     v = f32_to_bf16_bits(rng.standard_normal((N, heads, head_dim), dtype=np.float32))
     return out[0], out[1], v, cu_seqlens_of(seg_lens)
+
+
+@dataclass(frozen=True)
+class QkvProjection:
+    """Shape of the DiT attention's input projection, the step that produces
+    this path's q, k, v: hidden size 5376 and 56 heads of 128 ("Day 0 Support
+    for MiniMax-H3 on AMD Instinct GPUs", section "The diffusion transformer
+    (DiT)"), rotary split (32, 48, 48) as for the attention workloads."""
+
+    hidden: int = 5376
+    heads: int = 56
+    head_dim: int = 128
+    split: tuple = (32, 48, 48)
+    theta: float = 10000.0
+
+    @property
+    def out_features(self) -> int:
+        return 3 * self.heads * self.head_dim
+
+
+QKV_PROJECTION = QkvProjection()
+
+
+def draw_linear_case(n_rows: int, k: int, out_features: int, seed: int):
+    """Activations and weights of one linear layer as bf16 bit patterns.
+
+    Recipe: ``numpy.random.default_rng(seed)``; x [n_rows, k] standard normal
+    float32 drawn in chunks of 16384 rows, then w [out_features, k] standard
+    normal float32 times 1/sqrt(k) (so every output is ~N(0, 1)), each rounded
+    to bf16 (round to nearest even).
+    """
+    rng = np.random.default_rng(seed)
+    x = _normal_bf16(rng, (n_rows, k))
+    w32 = rng.standard_normal((out_features, k), dtype=np.float32)
+    w32 *= np.float32(1.0 / np.sqrt(k))
+    return x, f32_to_bf16_bits(w32)

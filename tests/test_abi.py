@@ -133,3 +133,31 @@ def test_selftest_host_argument_errors():
     assert h3.h3_selftest_bounded_wait(0x10010, 256, 1000, 0) == h3.H3_ERR_WORKSPACE
     assert h3.h3_selftest_bounded_wait(0x10000, 128, 1000, 0) == h3.H3_ERR_WORKSPACE
     assert h3.h3_selftest_bounded_wait(0x10000, 256, 0, 0) == h3.H3_ERR_INVALID_ARG
+
+
+def _qkv(**over):
+    a = dict(x=0x10000, w=0x20000, q=0x30000, k=0x40000, v=0x50000, pos=0x60000,
+             rope=h3.rope_cfg((32, 48, 48), 1e4), N=300, K=256, H=2, D=128,
+             workspace=0x70000, workspace_bytes=256, stream=0)
+    a.update(over)
+    return h3.h3_qkv_rope_gemm(**a)
+
+
+def test_qkv_gemm_host_argument_errors():
+    # rejected before any CUDA call (no GPU needed)
+    assert _qkv(D=96) == h3.H3_ERR_UNSUPPORTED
+    assert _qkv(K=200) == h3.H3_ERR_INVALID_ARG          # K % 64 != 0
+    assert _qkv(K=0) == h3.H3_ERR_INVALID_ARG
+    assert _qkv(H=1, D=64, rope=h3.rope_cfg((16, 24, 24), 1e4)) == h3.H3_ERR_INVALID_ARG  # HD % 256
+    assert _qkv(H=3) == h3.H3_ERR_INVALID_ARG            # HD = 384
+    assert _qkv(H=0) == h3.H3_ERR_INVALID_ARG
+    assert _qkv(N=-1) == h3.H3_ERR_INVALID_ARG
+    assert _qkv(x=0) == h3.H3_ERR_INVALID_ARG
+    assert _qkv(v=0) == h3.H3_ERR_INVALID_ARG
+    assert _qkv(rope=h3.rope_cfg((32, 48, 46), 1e4)) == h3.H3_ERR_INVALID_ARG
+    assert _qkv(x=0x10008) == h3.H3_ERR_MISALIGNED
+    assert _qkv(k=0x40002) == h3.H3_ERR_MISALIGNED
+    assert _qkv(pos=0x60002) == h3.H3_ERR_MISALIGNED
+    assert _qkv(workspace=0) == h3.H3_ERR_WORKSPACE
+    assert _qkv(workspace=0x70080) == h3.H3_ERR_WORKSPACE
+    assert _qkv(workspace_bytes=255) == h3.H3_ERR_WORKSPACE
