@@ -423,6 +423,83 @@ def run_skip(args, wl, rank, world, local_rank):
     return 0
 
 
+def run_qkv(args, wl, rank, world, local_rank):
+    """The QKV projection with RoPE fused into its epilogue (h3_qkv_rope_gemm)
+    on the DiT's shape (hidden 5376 -> 3 x 56 heads x 128) over the tokens and
+    positions of workload ``wl``. Reports TFLOP/s (2 N K 3HD per call) against
+    the measured bf16 peaks, and the unfused alternative with the same
+    kernels: the projection without rotation followed by the standalone
+    rotary pass over q and k. Inputs (X alone is N*5376*2 bytes) exceed L2.
+    Single process only."""
+    import torch
+
+    import audio_diffusion_transformer_h3_b200 as h3
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    p = synth.QKV_PROJECTION
+    N, K, H, D = wl.n_tokens, p.hidden, p.heads, p.head_dim
+    x_bits, w_bits = synth.draw_linear_case(N, K, p.out_features, seed=rank_seed(90, rank))
+    pos, _ = h3.h3_build_positions(wl.segments)
+
+    def bf(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    x, w = bf(x_bits), bf(w_bits)
+    del x_bits, w_bits
+    dpos = torch.from_numpy(pos).to(dev)
+    out = tuple(torch.empty((N, H, D), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    def fused():
+        h3.qkv_rope_gemm_t(x, w, H, D, dpos, p.split, p.theta, out=out, workspace=ws,
+                           stream=stream)
+
+    def unfused():
+        h3.qkv_rope_gemm_t(x, w, H, D, None, None, out=out, workspace=ws, stream=stream)
+        h3.rope_apply_t(out[0], dpos, p.split, p.theta, out=out[0], stream=stream)
+        h3.rope_apply_t(out[1], dpos, p.split, p.theta, out=out[1], stream=stream)
+
+    with ClockSampler(str(local_rank)) as clocks:
+        ms = timed(fused)
+    assert h3.device_status_t(ws) == h3.H3_OK
+    ms_unfused = timed(unfused)
+    flops = 2.0 * N * K * p.out_features
+    achieved = flops / (ms * 1e-3) / 1e12
+    peaks = measured_peaks()
+    line = {"metric": "QKV projection with fused RoPE epilogue, TFLOP/s",
+            "value": achieved, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic (synth.draw_linear_case, x ~ N(0,1), "
+                                     "w ~ N(0,1/K); positions of the workload)",
+            "config": {"workload": f"qkv projection {N}x{K} -> 3x{H}x{D} "
+                                   f"({wl.name} workload tokens)",
+                       "tokens": N, "hidden": K, "heads": H, "head_dim": D,
+                       "l2": "inputs larger than L2 (no flush)"},
+            "roofline": {"bound": "tensor", "achieved": achieved,
+                         "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_sustained"],
+                         "peak_kind": f"bf16 dense, sustained ({peaks['source']})",
+                         "frac_of_burst": achieved / peaks["bf16"]},
+            "unfused_ms": ms_unfused, "fusion_speedup": ms_unfused / ms,
+            "gpu_launches": args.steps, "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,6 +512,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--skip-threshold", type=float, default=None,
                     help="time the skip-softmax variant on frame-group inputs instead")
+    ap.add_argument("--qkv-proj", action="store_true",
+                    help="time the QKV projection with the fused RoPE epilogue instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -448,6 +527,8 @@ def main():
         return run_reference(args, wl, rank, world)
     if args.skip_threshold is not None:
         return run_skip(args, wl, rank, world, local_rank)
+    if args.qkv_proj:
+        return run_qkv(args, wl, rank, world, local_rank)
 
     if world > 1:
         import datetime
