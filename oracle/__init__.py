@@ -24,6 +24,9 @@ What it computes, and the passages it follows:
 * ``qkv_rope``    -- the qkv projection with RoPE applied to q and k in its
   epilogue ("MiniMax-H3 Reference" Space README, section "AoTI-compiled
   blocks": rotary epilogues around the block's matmuls).
+* ``sage``        -- the lossy SAGE-style FP8 attention: e4m3 Q/K with
+  per-token and per-16-key scales, FP8 P and V ("MiniMax H3" vLLM-Omni
+  recipe, section "Attention Backends"), with its e4m3 codec.
 
 Readings where the pages say nothing (pair layout, frequency schedule,
 audio-token clock, reference layout) are listed in the design notes of the
@@ -45,3 +48,11 @@ from .attention import (  # noqa: F401
 )
 from .skip_softmax import attention_skip_ref, attention_skip_rows_ref  # noqa: F401
 from .qkv_rope import qkv_rope_ref  # noqa: F401
+from .sage import (  # noqa: F401
+    e4m3_decode,
+    e4m3_encode,
+    e4m3_round,
+    sage_quantize,
+    sage_attention_ref,
+    sage_attention_rows_ref,
+)
