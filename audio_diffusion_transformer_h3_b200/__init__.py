@@ -72,6 +72,12 @@ _lib.h3_varlen_attn_fwd_skip.argtypes = [_P, _P, _P, _P, _P, _P, _c.c_int32, _c.
                                          h3_rope_cfg, _c.c_int64, _c.c_int32, _c.c_int32,
                                          _c.c_float, _c.c_float, _P, _c.c_size_t, _P]
 _lib.h3_varlen_attn_fwd_skip.restype = _c.c_int
+_lib.h3_sage_workspace_size.argtypes = [_c.c_int64, _c.c_int32, _c.c_int32, _c.c_int32]
+_lib.h3_sage_workspace_size.restype = _c.c_size_t
+_lib.h3_varlen_attn_fwd_sage.argtypes = [_P, _P, _P, _P, _P, _P, _c.c_int32, _c.c_int32, _P,
+                                         h3_rope_cfg, _c.c_int64, _c.c_int32, _c.c_int32,
+                                         _c.c_float, _P, _c.c_size_t, _P]
+_lib.h3_varlen_attn_fwd_sage.restype = _c.c_int
 _lib.h3_qkv_rope_gemm.argtypes = [_P, _P, _P, _P, _P, _P, h3_rope_cfg, _c.c_int64, _c.c_int32,
                                   _c.c_int32, _c.c_int32, _P, _c.c_size_t, _P]
 _lib.h3_qkv_rope_gemm.restype = _c.c_int
@@ -88,7 +94,7 @@ _lib.h3_last_cuda_error.restype = _c.c_int32
 
 EXPORTED = ("h3_segment_tokens", "h3_build_positions", "h3_rope_apply", "h3_workspace_size",
             "h3_varlen_attn_fwd", "h3_varlen_attn_fwd_skip", "h3_read_skip_count",
-            "h3_qkv_rope_gemm",
+            "h3_qkv_rope_gemm", "h3_sage_workspace_size", "h3_varlen_attn_fwd_sage",
             "h3_varlen_attn_fwd_static", "h3_selftest_bounded_wait",
             "h3_read_device_status", "h3_status_string", "h3_last_cuda_error")
 
@@ -154,6 +160,19 @@ def h3_varlen_attn_fwd_skip(q: int, k: int, v: int, o: int, lse: int, cu_seqlens
     return int(_lib.h3_varlen_attn_fwd_skip(q, k, v, o, lse, cu_seqlens, nseg, max_seqlen, pos,
                                             rope, N, H, D, softmax_scale, skip_threshold,
                                             workspace, workspace_bytes, stream))
+
+
+def h3_sage_workspace_size(N: int, H: int, D: int, nseg: int) -> int:
+    return int(_lib.h3_sage_workspace_size(N, H, D, nseg))
+
+
+def h3_varlen_attn_fwd_sage(q: int, k: int, v: int, o: int, lse: int, cu_seqlens: int,
+                            nseg: int, max_seqlen: int, pos: int, rope: h3_rope_cfg, N: int,
+                            H: int, D: int, softmax_scale: float, workspace: int,
+                            workspace_bytes: int, stream: int) -> int:
+    return int(_lib.h3_varlen_attn_fwd_sage(q, k, v, o, lse, cu_seqlens, nseg, max_seqlen, pos,
+                                            rope, N, H, D, softmax_scale, workspace,
+                                            workspace_bytes, stream))
 
 
 def h3_qkv_rope_gemm(x: int, w: int, q: int, k: int, v: int, pos: int, rope: h3_rope_cfg,
@@ -326,6 +345,65 @@ def qkv_rope_gemm_t(x, w, heads: int, head_dim: int, pos=None, split=None,
                           head_dim, workspace.data_ptr(), workspace.numel(), _stream(stream))
     _check(st, "h3_qkv_rope_gemm")
     return q, k, v
+
+
+def sage_workspace_for(N: int, H: int, D: int, nseg: int, device=None):
+    import torch
+    n = h3_sage_workspace_size(N, H, D, nseg)
+    if n == 0:
+        raise ValueError("the SAGE variant supports head dim 128 only")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def sage_workspace_views(workspace, N: int, H: int, nseg: int) -> dict:
+    """Views of the regions h3_varlen_attn_fwd_sage leaves in its workspace
+    (layout of h3_sage_workspace_size in include/h3attn.h): q8, k8, v8 uint8
+    [N, H, 128]; s_q, s_k float32 [H, N]; v_amax, s_v float32 [nseg, H, 128]."""
+    import torch
+
+    def up(x):
+        return (x + 255) // 256 * 256
+    codes, scales, vsc = up(N * H * 128), up(N * H * 4), up(nseg * H * 128 * 4)
+    off = {"q8": 256}
+    off["k8"] = off["q8"] + codes
+    off["v8"] = off["k8"] + codes
+    off["s_q"] = off["v8"] + codes
+    off["s_k"] = off["s_q"] + scales
+    off["v_amax"] = off["s_k"] + scales
+    off["s_v"] = off["v_amax"] + vsc
+    out = {}
+    for name in ("q8", "k8", "v8"):
+        out[name] = workspace[off[name]:off[name] + N * H * 128].view(N, H, 128)
+    for name in ("s_q", "s_k"):
+        out[name] = workspace[off[name]:off[name] + N * H * 4].view(torch.float32).view(H, N)
+    for name in ("v_amax", "s_v"):
+        out[name] = workspace[off[name]:off[name] + nseg * H * 512].view(torch.float32) \
+            .view(nseg, H, 128)
+    return out
+
+
+def varlen_attn_fwd_sage_t(q, k, v, cu_seqlens, max_seqlen: int, pos=None, split=None,
+                           theta: float = 10000.0, softmax_scale: Optional[float] = None,
+                           out=None, return_lse: bool = False, workspace=None, stream=None):
+    """SAGE-style FP8 variant through h3_varlen_attn_fwd_sage (head dim 128)."""
+    import torch
+    _thd(q, "q"); _thd(k, "k"); _thd(v, "v")
+    N, H, D = q.shape
+    nseg = int(cu_seqlens.numel()) - 1
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((H, N), dtype=torch.float32, device=q.device) if return_lse else None
+    if workspace is None:
+        workspace = sage_workspace_for(N, H, D, nseg, q.device)
+    scale = (1.0 / math.sqrt(D)) if softmax_scale is None else float(softmax_scale)
+    rope = rope_cfg(split, theta) if pos is not None else h3_rope_cfg(0, 0, 0, 0.0)
+    st = h3_varlen_attn_fwd_sage(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr() if lse is not None else 0,
+                                 cu_seqlens.data_ptr(), nseg, int(max_seqlen),
+                                 pos.data_ptr() if pos is not None else 0, rope, N, H, D, scale,
+                                 workspace.data_ptr(), workspace.numel(), _stream(stream))
+    _check(st, "h3_varlen_attn_fwd_sage")
+    return (out, lse) if return_lse else out
 
 
 def skip_count_t(workspace, stream=None) -> int:

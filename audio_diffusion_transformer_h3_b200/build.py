@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libh3attn.so")
 
 SOURCES = [os.path.join(CSRC, "h3attn.cu"), os.path.join(CSRC, "h3attn_static.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("sm100.cuh", "rope.cuh", "attn_fwd.cuh", "qkv_gemm.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("sm100.cuh", "rope.cuh", "attn_fwd.cuh", "attn_sage.cuh", "qkv_gemm.cuh")] + [
     os.path.join(INCLUDE, "h3attn.h")]
 
 

@@ -3,7 +3,7 @@
 // Host side only: argument validation, the rotary frequency table, TMA
 // descriptors, launches on the caller's stream, and the host position
 // builder. Every step of the device path runs in the kernels of
-// rope.cuh, attn_fwd.cuh and qkv_gemm.cuh; nothing here computes on the host except
+// rope.cuh, attn_fwd.cuh, attn_sage.cuh and qkv_gemm.cuh; nothing here computes on the host except
 // positions (which the pages place on the host: "MiniMax H3 on Moore Threads
 // MUSA", section "MUSA validation").
 #include <cuda.h>
@@ -16,6 +16,7 @@
 
 #include "h3attn.h"
 #include "attn_fwd.cuh"
+#include "attn_sage.cuh"
 #include "qkv_gemm.cuh"
 #include "rope.cuh"
 
@@ -97,6 +98,9 @@ h3_status device_info(DeviceInfo **out) {
                 (e = cudaFuncSetAttribute(h3::attn_fwd_kernel<64, true>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           h3::AttnCfg<64>::SMEM_BYTES)) != cudaSuccess ||
+                (e = cudaFuncSetAttribute(h3::attn_sage_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          h3::SageCfg::SMEM_BYTES)) != cudaSuccess ||
                 (e = cudaFuncSetAttribute(h3::qkv_rope_gemm_kernel<128>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           h3::QkvCfg::SMEM_BYTES)) != cudaSuccess ||
@@ -168,6 +172,44 @@ h3_status make_2d_map(CUtensorMap *map, const void *base, int64_t rows, int64_t 
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
     return H3_OK;
+}
+
+// TMA map over an e4m3 [N, H, 128] tensor: dims (128, H, N) bytes, box
+// (128, 1, 128), 128-byte swizzle, zero fill out of bounds.
+h3_status make_u8_thd_map(CUtensorMap *map, const void *base, int64_t N, int H) {
+    EncodeTiledFn enc = encode_tiled();
+    if (enc == nullptr) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(N)};
+    const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(H) * 128};
+    const cuuint32_t box[3] = {128, 1, 128};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    return H3_OK;
+}
+
+// Byte offsets of the SAGE workspace regions (see h3_sage_workspace_size).
+struct SageLayout {
+    size_t q8, k8, v8, s_q, s_k, v_amax, s_v, total;
+};
+
+SageLayout sage_layout(int64_t N, int32_t H, int32_t nseg) {
+    SageLayout L;
+    const size_t codes = round_up(static_cast<size_t>(N) * H * 128, 256);
+    const size_t scales = round_up(static_cast<size_t>(N) * H * 4, 256);
+    const size_t vsc = round_up(static_cast<size_t>(nseg) * H * 128 * 4, 256);
+    L.q8 = kStatusBytes;
+    L.k8 = L.q8 + codes;
+    L.v8 = L.k8 + codes;
+    L.s_q = L.v8 + codes;
+    L.s_k = L.s_q + scales;
+    L.v_amax = L.s_k + scales;
+    L.s_v = L.v_amax + vsc;
+    L.total = L.s_v + vsc;
+    return L;
 }
 
 h3_status launch_rope(const void *x, void *out, const float *pos, int64_t N, int H, int D,
@@ -433,6 +475,97 @@ h3_status h3_qkv_rope_gemm(const void *x, const void *w, void *q, void *k, void 
         h3::qkv_rope_gemm_kernel<128><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tx, tw, p);
     else
         h3::qkv_rope_gemm_kernel<64><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tx, tw, p);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? H3_OK : cuda_fail(e);
+}
+
+size_t h3_sage_workspace_size(int64_t N, int32_t H, int32_t D, int32_t nseg) {
+    if (N < 0 || H < 0 || D != 128 || nseg < 0) return 0;
+    return sage_layout(N, H, nseg).total;
+}
+
+h3_status h3_varlen_attn_fwd_sage(const void *q, const void *k, const void *v, void *o,
+                                  float *lse, const int32_t *cu_seqlens, int32_t nseg,
+                                  int32_t max_seqlen, const float *pos, h3_rope_cfg rope,
+                                  int64_t N, int32_t H, int32_t D, float softmax_scale,
+                                  void *workspace, size_t workspace_bytes, h3_stream_t stream) {
+    if (N < 0 || N > INT32_MAX - 1 || H < 1 || H > 65535 || nseg < 1 || nseg > 65535)
+        return H3_ERR_INVALID_ARG;
+    if (D != 128) return H3_ERR_UNSUPPORTED;
+    if (!std::isfinite(softmax_scale) || softmax_scale < 0.0f) return H3_ERR_INVALID_ARG;
+    if (cu_seqlens == nullptr) return H3_ERR_INVALID_ARG;
+    if (N > 0 && (q == nullptr || k == nullptr || v == nullptr || o == nullptr))
+        return H3_ERR_INVALID_ARG;
+    if (N > 0 && (max_seqlen < 1 || max_seqlen > N)) return H3_ERR_INVALID_ARG;
+    h3::RopeTable rt;
+    std::memset(&rt, 0, sizeof(rt));
+    if (pos != nullptr && !make_rope_table(rope, D, &rt)) return H3_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(pos, 4) || !aligned(lse, 4) || !aligned(cu_seqlens, 4))
+        return H3_ERR_MISALIGNED;
+    const SageLayout lay = sage_layout(N, H, nseg);
+    if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < lay.total)
+        return H3_ERR_WORKSPACE;
+
+    DeviceInfo *d = nullptr;
+    h3_status st = device_info(&d);
+    if (st != H3_OK) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int *status = reinterpret_cast<int *>(ws);
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), cs);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(ws + lay.v_amax, 0, static_cast<size_t>(nseg) * H * 128 * 4, cs);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (N == 0) return H3_OK;
+
+    h3::SageQuantParams qp;
+    qp.q = static_cast<const __nv_bfloat16 *>(q);
+    qp.k = static_cast<const __nv_bfloat16 *>(k);
+    qp.v = static_cast<const __nv_bfloat16 *>(v);
+    qp.cu_seqlens = cu_seqlens;
+    qp.pos = pos;
+    qp.q8 = ws + lay.q8;
+    qp.k8 = ws + lay.k8;
+    qp.v8 = ws + lay.v8;
+    qp.s_q = reinterpret_cast<float *>(ws + lay.s_q);
+    qp.s_k = reinterpret_cast<float *>(ws + lay.s_k);
+    qp.v_amax = reinterpret_cast<unsigned *>(ws + lay.v_amax);
+    qp.s_v = reinterpret_cast<float *>(ws + lay.s_v);
+    qp.status = status;
+    qp.nseg = nseg;
+    qp.max_seqlen = max_seqlen;
+    qp.N = static_cast<int32_t>(N);
+    qp.H = H;
+    qp.rope = rt;
+    const dim3 qgrid(static_cast<unsigned>((max_seqlen + 127) / 128), static_cast<unsigned>(H),
+                     static_cast<unsigned>(nseg));
+    h3::sage_vamax_kernel<<<qgrid, 256, 0, cs>>>(qp);
+    h3::sage_quant_kernel<<<qgrid, 256, 0, cs>>>(qp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+
+    CUtensorMap tq, tk, tv;
+    if ((st = make_u8_thd_map(&tq, qp.q8, N, H)) != H3_OK) return st;
+    if ((st = make_u8_thd_map(&tk, qp.k8, N, H)) != H3_OK) return st;
+    if ((st = make_u8_thd_map(&tv, qp.v8, N, H)) != H3_OK) return st;
+    h3::SageAttnParams ap;
+    ap.cu_seqlens = cu_seqlens;
+    ap.s_q = qp.s_q;
+    ap.s_k = qp.s_k;
+    ap.s_v = qp.s_v;
+    ap.o = static_cast<__nv_bfloat16 *>(o);
+    ap.lse = lse;
+    ap.status = status;
+    ap.nseg = nseg;
+    ap.max_seqlen = max_seqlen;
+    ap.N = static_cast<int32_t>(N);
+    ap.H = H;
+    ap.scale_log2 = softmax_scale * 1.4426950408889634f;
+    const dim3 grid(static_cast<unsigned>((max_seqlen + 255) / 256), static_cast<unsigned>(H),
+                    static_cast<unsigned>(nseg));
+    h3::attn_sage_kernel<<<grid, h3::SageCfg::THREADS, h3::SageCfg::SMEM_BYTES, cs>>>(tq, tk,
+                                                                                     tv, ap);
     e = cudaGetLastError();
     return e == cudaSuccess ? H3_OK : cuda_fail(e);
 }

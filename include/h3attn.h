@@ -167,6 +167,41 @@ h3_status h3_varlen_attn_fwd_skip(const void *q, const void *k, const void *v, v
                                   float skip_threshold, void *workspace, size_t workspace_bytes,
                                   h3_stream_t stream);
 
+/* Bytes of device workspace h3_varlen_attn_fwd_sage needs (0 if D != 128 or
+ * a size is negative). Layout, each region starting on a 256-byte boundary
+ * in this order: the 256-byte status block; q8, k8, v8 (e4m3 codes, [N, H,
+ * 128] bytes each, regions of round_up(N*H*128, 256)); s_q, s_k (fp32
+ * dequantisation scales [H, N], s_k repeated for every token of its 16-key
+ * block; regions of round_up(N*H*4, 256)); v_amax (fp32 [nseg, H, 128], max
+ * |v| per segment, head and channel) and s_v (fp32 [nseg, H, 128], v_amax /
+ * 448; regions of round_up(nseg*H*128*4, 256)). A call leaves its quantised
+ * tensors and scales there. */
+size_t h3_sage_workspace_size(int64_t N, int32_t H, int32_t D, int32_t nseg);
+
+/* SAGE-style FP8 variant of h3_varlen_attn_fwd (lossy). "MiniMax H3"
+ * vLLM-Omni recipe, section "Attention Backends": Q and K in fp8_e4m3 with
+ * q_block_size 1 and k_block_size 16, P and V in FP8. Reading used here
+ * (conversions to e4m3 round to nearest even and saturate to +-448):
+ *   Q~ = RoPE(q), K~ = RoPE(k) in fp32 (pos NULL: no rotation);
+ *   Q: per (token, head) a = max|Q~|, codes e4m3(Q~ * (448/a)), s_q = a/448;
+ *   K: per (16-key block from the segment start, head), same formulas;
+ *   V: per (segment, head, channel), same formulas over the segment's tokens;
+ *   scores x = (q8.k8) s_q s_k softmax_scale log2(e); online softmax over key
+ *   tiles of 128 from the segment start, the running max m raised whenever a
+ *   tile raises it; P8 = e4m3(448 * 2^(x - m)); the row sum l adds the
+ *   unquantised 448 * 2^(x - m); O = s_v (P8 V8) / l, rounded to bf16;
+ *   LSE = (m + log2(l / 448)) ln 2.
+ * Arguments as h3_varlen_attn_fwd except: D must be 128 (else
+ * H3_ERR_UNSUPPORTED) and the workspace is >= h3_sage_workspace_size bytes.
+ * Launches: a V max pass, a quantisation pass (RoPE fused), the FP8 attention
+ * kernel. Invalid cu_seqlens set H3_ERR_BAD_SEQLENS without any access
+ * outside [0, N). Deterministic. */
+h3_status h3_varlen_attn_fwd_sage(const void *q, const void *k, const void *v, void *o,
+                                  float *lse, const int32_t *cu_seqlens, int32_t nseg,
+                                  int32_t max_seqlen, const float *pos, h3_rope_cfg rope,
+                                  int64_t N, int32_t H, int32_t D, float softmax_scale,
+                                  void *workspace, size_t workspace_bytes, h3_stream_t stream);
+
 /* Waits for `stream`, then writes to *count the number of (32-row block, key
  * tile) pairs the last h3_varlen_attn_fwd_skip call on `workspace` skipped.
  * H3_ERR_WORKSPACE / H3_ERR_INVALID_ARG on null pointers, H3_ERR_CUDA if the

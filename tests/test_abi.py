@@ -161,3 +161,28 @@ def test_qkv_gemm_host_argument_errors():
     assert _qkv(workspace=0) == h3.H3_ERR_WORKSPACE
     assert _qkv(workspace=0x70080) == h3.H3_ERR_WORKSPACE
     assert _qkv(workspace_bytes=255) == h3.H3_ERR_WORKSPACE
+
+
+def test_sage_workspace_layout_and_host_errors():
+    # status | q8 k8 v8 | s_q s_k | v_amax s_v, every region 256-aligned
+    N, H, nseg = 1000, 3, 2
+    up = lambda x: (x + 255) // 256 * 256
+    assert h3.h3_sage_workspace_size(N, H, 128, nseg) == \
+        256 + 3 * up(N * H * 128) + 2 * up(N * H * 4) + 2 * up(nseg * H * 512)
+    assert h3.h3_sage_workspace_size(N, H, 64, nseg) == 0
+    a = dict(q=0x10000, k=0x20000, v=0x30000, o=0x40000, lse=0, cu_seqlens=0x50000, nseg=2,
+             max_seqlen=80, pos=0, rope=h3.h3_rope_cfg(0, 0, 0, 0.0), N=160, H=2, D=128,
+             softmax_scale=0.125, workspace=0x70000, workspace_bytes=1 << 24, stream=0)
+
+    def call(**over):
+        b = dict(a)
+        b.update(over)
+        return h3.h3_varlen_attn_fwd_sage(**b)
+    assert call(D=64) == h3.H3_ERR_UNSUPPORTED
+    assert call(nseg=0) == h3.H3_ERR_INVALID_ARG
+    assert call(softmax_scale=-1.0) == h3.H3_ERR_INVALID_ARG
+    assert call(max_seqlen=0) == h3.H3_ERR_INVALID_ARG
+    assert call(pos=0x60000, rope=h3.rope_cfg((32, 48, 46), 1e4)) == h3.H3_ERR_INVALID_ARG
+    assert call(q=0x10008) == h3.H3_ERR_MISALIGNED
+    assert call(workspace_bytes=1000) == h3.H3_ERR_WORKSPACE
+    assert call(workspace=0x70010) == h3.H3_ERR_WORKSPACE
