@@ -10,9 +10,13 @@
 //   K: one scale per (16-key block, head), blocks from the segment start;
 //   V: one scale per (segment, head, channel);
 //   scores x = (q8 . k8) * s_q * s_k * softmax_scale * log2(e);
-//   online softmax over key tiles of 128 with the running max m updated
-//   whenever a tile raises it; P8 = e4m3(448 * 2^(x - m)); the row sum l adds
-//   the unquantised 448 * 2^(x - m); O = s_v * (P8 V8) / l.
+//   online softmax over key tiles of 128 with a lazily updated reference max
+//   m: m is raised to the running max only when a tile's max exceeds it by
+//   more than 2 (log2 units), so 2^(x - m) <= 4; P8 = e4m3(112 * 2^(x - m))
+//   (<= 448); the row sum l adds the unquantised 112 * 2^(x - m);
+//   O = s_v * (P8 V8) / l. Exponentials: three quarters on MUFU
+//   (ex2.approx), one quarter on the FMA pipe (exp2_fma, relative error
+//   below 2e-4), which shares the load between the two pipes.
 // e4m3 conversions round to nearest even and saturate to +-448
 // (cvt.rn.satfinite).
 //
@@ -20,7 +24,8 @@
 //   sage_vamax_kernel   per (segment, head, channel) max |v| (atomicMax on the
 //                       bit patterns of non-negative floats);
 //   sage_quant_kernel   RoPE + quantisation of q, k, v into e4m3 codes and
-//                       scales; one warp per 16-token block, lane = 4 channels;
+//                       scales; one CTA per 16-token block (all heads, the
+//                       block's rotary table computed once), lane = 4 channels;
 //   attn_sage_kernel    the attention kernel of attn_fwd.cuh in FP8: the same
 //                       warp roles, barriers and TMEM plan, tcgen05.mma
 //                       kind::f8f6f4 for S = Q8 K8^T (A, B K-major in shared
@@ -39,7 +44,8 @@
 namespace h3 {
 
 constexpr float kE4m3Max = 448.0f;
-constexpr float kLog2E4m3Max = 8.807354922057604f;  // log2(448)
+constexpr float kLazyLog2 = 2.0f;                  // lazy max threshold (log2 units)
+constexpr float kLog2PScale = 6.807354922057604f;  // log2(448 / 2^kLazyLog2) = log2(112)
 
 struct SageQuantParams {
     const __nv_bfloat16 *q, *k, *v;   // [N, H, 128]
@@ -124,100 +130,125 @@ __global__ void __launch_bounds__(256) sage_vamax_kernel(const SageQuantParams p
     }
 }
 
-// grid (ceil(max_seqlen / 128), H, nseg), 256 threads. Warp w quantises the
-// 16-token block [t0 + 16w, t0 + 16w + 16) of the segment (the K scale block);
-// lane l holds channels 4l .. 4l+3 (rotary pairs 2l and 2l+1).
+// grid (ceil(max_seqlen / 16), nseg), 256 threads. A CTA takes one 16-token
+// block of a segment (the K scale block, counted from the segment start) for
+// every head: it first builds the block's (cos, sin) table (16 tokens x 64
+// pairs) in shared memory, then warp w quantises heads w, w + 8, ...; lane l
+// holds channels 4l .. 4l+3 (rotary pairs 2l and 2l+1). All 48 row fragments
+// of a (block, head) are loaded before the first store.
 __global__ void __launch_bounds__(256) sage_quant_kernel(const SageQuantParams p) {
-    const int seg = blockIdx.z, head = blockIdx.y, tile = blockIdx.x;
+    __shared__ float4 cs[16][32];   // per token and lane: (cos, sin) of pairs 2l, 2l+1
+    const int seg = blockIdx.y, blk = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int a, e;
     if (!sage_segment(p.cu_seqlens, seg, p.N, p.max_seqlen, p.status, a, e)) return;
-    const int b0 = a + tile * 128 + warp * 16;
-    const int64_t vrow = (static_cast<int64_t>(seg) * p.H + head) * 128 + lane * 4;
-    // V: per-channel inverse scales of this segment and head
-    float vinv[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float am = __uint_as_float(p.v_amax[vrow + i]);
-        vinv[i] = am > 0.0f ? __fdiv_rn(kE4m3Max, am) : 0.0f;
-        if (tile == 0 && warp == 0) p.s_v[vrow + i] = __fdiv_rn(am, kE4m3Max);
+    const int b0 = a + blk * 16;
+    if (blk == 0) {
+        // per-channel dequantisation scales of V (also for an empty segment)
+        for (int i = threadIdx.x; i < p.H * 128; i += 256) {
+            const int64_t at = static_cast<int64_t>(seg) * p.H * 128 + i;
+            p.s_v[at] = __fdiv_rn(__uint_as_float(p.v_amax[at]), kE4m3Max);
+        }
     }
     if (b0 >= e) return;
     const int n = min(16, e - b0);
-    const int pr0 = 2 * lane, pr1 = 2 * lane + 1;
-    float kx[16][4];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) kx[j][i] = 0.0f;
-        if (j >= n) continue;
-        const int t = b0 + j;
-        const int64_t off = (static_cast<int64_t>(t) * p.H + head) * 128 + lane * 4;
+    for (int i = threadIdx.x; i < 16 * 32; i += 256) {
+        const int j = i >> 5, l = i & 31;
         float c0 = 1.0f, s0 = 0.0f, c1 = 1.0f, s1 = 0.0f;
-        if (p.pos != nullptr) {
-            rope_cos_sin(p.pos[static_cast<int64_t>(t) * 3 + rope_axis(p.rope, pr0)],
-                         p.rope.inv_freq[pr0], c0, s0);
-            rope_cos_sin(p.pos[static_cast<int64_t>(t) * 3 + rope_axis(p.rope, pr1)],
-                         p.rope.inv_freq[pr1], c1, s1);
+        if (p.pos != nullptr && j < n) {
+            const float *pp = p.pos + static_cast<int64_t>(b0 + j) * 3;
+            rope_cos_sin(pp[rope_axis(p.rope, 2 * l)], p.rope.inv_freq[2 * l], c0, s0);
+            rope_cos_sin(pp[rope_axis(p.rope, 2 * l + 1)], p.rope.inv_freq[2 * l + 1], c1, s1);
         }
-        // Q: rotate, one scale for the token
-        {
-            const uint2 u = *reinterpret_cast<const uint2 *>(p.q + off);
-            float x[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
-                          __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
-            if (p.pos != nullptr) {
-                rope_rotate(x[0], x[1], c0, s0, x[0], x[1]);
-                rope_rotate(x[2], x[3], c1, s1, x[2], x[3]);
-            }
-            const float lm = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
-            const float am = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(lm)));
-            const float inv = am > 0.0f ? __fdiv_rn(kE4m3Max, am) : 0.0f;
-            *reinterpret_cast<uint32_t *>(p.q8 + off) =
-                e4m3x4(__fmul_rn(x[0], inv), __fmul_rn(x[1], inv), __fmul_rn(x[2], inv),
-                       __fmul_rn(x[3], inv));
-            if (lane == 0) p.s_q[static_cast<int64_t>(head) * p.N + t] = __fdiv_rn(am, kE4m3Max);
-        }
-        // K: rotate, keep for the block scale
-        {
-            const uint2 u = *reinterpret_cast<const uint2 *>(p.k + off);
-            float x[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
-                          __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
-            if (p.pos != nullptr) {
-                rope_rotate(x[0], x[1], c0, s0, x[0], x[1]);
-                rope_rotate(x[2], x[3], c1, s1, x[2], x[3]);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) kx[j][i] = x[i];
-        }
-        // V: per-channel scales
-        {
-            const uint2 u = *reinterpret_cast<const uint2 *>(p.v + off);
-            const float x[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
-                                __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
-            *reinterpret_cast<uint32_t *>(p.v8 + off) =
-                e4m3x4(__fmul_rn(x[0], vinv[0]), __fmul_rn(x[1], vinv[1]),
-                       __fmul_rn(x[2], vinv[2]), __fmul_rn(x[3], vinv[3]));
-        }
+        cs[j][l] = make_float4(c0, s0, c1, s1);
     }
-    // K block scale over the block's tokens and channels
-    float lm = 0.0f;
+    __syncthreads();
+    const bool rotate = p.pos != nullptr;
+    for (int head = warp; head < p.H; head += 8) {
+        auto row = [&](int j) {
+            return (static_cast<int64_t>(b0 + j) * p.H + head) * 128 + lane * 4;
+        };
+        uint2 qraw[16], kraw[16], vraw[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
+        for (int j = 0; j < 16; ++j) {
+            const bool in = j < n;
+            kraw[j] = in ? __ldg(reinterpret_cast<const uint2 *>(p.k + row(j))) : make_uint2(0, 0);
+            qraw[j] = in ? __ldg(reinterpret_cast<const uint2 *>(p.q + row(j))) : make_uint2(0, 0);
+            vraw[j] = in ? __ldg(reinterpret_cast<const uint2 *>(p.v + row(j))) : make_uint2(0, 0);
+        }
+        const int64_t vrow = (static_cast<int64_t>(seg) * p.H + head) * 128 + lane * 4;
+        float vinv[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) lm = fmaxf(lm, fabsf(kx[j][i]));
-    const float am = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(lm)));
-    const float inv = am > 0.0f ? __fdiv_rn(kE4m3Max, am) : 0.0f;
-    const float sk = __fdiv_rn(am, kE4m3Max);
+        for (int i = 0; i < 4; ++i) {
+            const float am = __uint_as_float(p.v_amax[vrow + i]);
+            vinv[i] = am > 0.0f ? __fdiv_rn(kE4m3Max, am) : 0.0f;
+        }
+        float kx[16][4];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        if (j >= n) continue;
-        const int t = b0 + j;
-        const int64_t off = (static_cast<int64_t>(t) * p.H + head) * 128 + lane * 4;
-        *reinterpret_cast<uint32_t *>(p.k8 + off) =
-            e4m3x4(__fmul_rn(kx[j][0], inv), __fmul_rn(kx[j][1], inv), __fmul_rn(kx[j][2], inv),
-                   __fmul_rn(kx[j][3], inv));
+        for (int j = 0; j < 16; ++j) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) kx[j][i] = 0.0f;
+            if (j >= n) continue;
+            const int t = b0 + j;
+            const int64_t off = row(j);
+            const float4 c = cs[j][lane];
+            // Q: rotate, one scale for the token
+            {
+                const uint2 u = qraw[j];
+                float x[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                              __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
+                if (rotate) {
+                    rope_rotate(x[0], x[1], c.x, c.y, x[0], x[1]);
+                    rope_rotate(x[2], x[3], c.z, c.w, x[2], x[3]);
+                }
+                const float lm = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+                const float am = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(lm)));
+                const float inv = am > 0.0f ? __fdiv_rn(kE4m3Max, am) : 0.0f;
+                *reinterpret_cast<uint32_t *>(p.q8 + off) =
+                    e4m3x4(__fmul_rn(x[0], inv), __fmul_rn(x[1], inv), __fmul_rn(x[2], inv),
+                           __fmul_rn(x[3], inv));
+                if (lane == 0) p.s_q[static_cast<int64_t>(head) * p.N + t] = __fdiv_rn(am, kE4m3Max);
+            }
+            // K: rotate, keep for the block scale
+            {
+                const uint2 u = kraw[j];
+                float x[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                              __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
+                if (rotate) {
+                    rope_rotate(x[0], x[1], c.x, c.y, x[0], x[1]);
+                    rope_rotate(x[2], x[3], c.z, c.w, x[2], x[3]);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) kx[j][i] = x[i];
+            }
+            // V: per-channel scales
+            {
+                const uint2 u = vraw[j];
+                const float x[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                                    __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
+                *reinterpret_cast<uint32_t *>(p.v8 + off) =
+                    e4m3x4(__fmul_rn(x[0], vinv[0]), __fmul_rn(x[1], vinv[1]),
+                           __fmul_rn(x[2], vinv[2]), __fmul_rn(x[3], vinv[3]));
+            }
+        }
+        // K block scale over the block's tokens and channels
+        float lm = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) lm = fmaxf(lm, fabsf(kx[j][i]));
+        const float am = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(lm)));
+        const float inv = am > 0.0f ? __fdiv_rn(kE4m3Max, am) : 0.0f;
+        const float sk = __fdiv_rn(am, kE4m3Max);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            if (j >= n) continue;
+            *reinterpret_cast<uint32_t *>(p.k8 + row(j)) =
+                e4m3x4(__fmul_rn(kx[j][0], inv), __fmul_rn(kx[j][1], inv),
+                       __fmul_rn(kx[j][2], inv), __fmul_rn(kx[j][3], inv));
+        }
+        if (lane < n) p.s_k[static_cast<int64_t>(head) * p.N + b0 + lane] = sk;
     }
-    if (lane < n) p.s_k[static_cast<int64_t>(head) * p.N + b0 + lane] = sk;
 }
 
 // ------------------------------------------------------------ FP8 attention
@@ -504,13 +535,13 @@ __global__ void __launch_bounds__(320, 1)
             float f = 1.0f;
             if (j == 0) {
                 m_used = mx;
-            } else if (mx > m_used) {
+            } else if (mx > m_used + kLazyLog2) {
                 need = true;
                 f = ex2_approx(m_used - mx);
                 l *= f;
                 m_used = mx;
             }
-            const float nm = kLog2E4m3Max - m_used;   // 448 * 2^(x - m) = 2^(x - m + log2 448)
+            const float nm = kLog2PScale - m_used;    // 112 * 2^(x - m) = 2^(x - m + log2 112)
             float lq[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             uint32_t pk[32];
             if (partial) {
@@ -533,7 +564,9 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int c = 4 * w + i;
-                        pv[i] = ex2_approx(fmaf(__uint_as_float(s[c]), cb[c >> 4], nm));
+                        const float y = fmaf(__uint_as_float(s[c]), cb[c >> 4], nm);
+                        // words 6 and 7 of every 8 on the FMA pipe, the rest on MUFU
+                        pv[i] = (w & 7) >= 6 ? exp2_fma(y) : ex2_approx(y);
                     }
                     lq[w & 3] += (pv[0] + pv[1]) + (pv[2] + pv[3]);
                     pk[w] = e4m3x4(pv[0], pv[1], pv[2], pv[3]);
@@ -593,7 +626,7 @@ __global__ void __launch_bounds__(320, 1)
             }
             if (valid && p.lse != nullptr)
                 p.lse[static_cast<int64_t>(head) * p.N + qrow] =
-                    (m_used + log2f(l) - kLog2E4m3Max) * 0.69314718055994530942f;
+                    (m_used + log2f(l) - kLog2PScale) * 0.69314718055994530942f;
         }
     }
 

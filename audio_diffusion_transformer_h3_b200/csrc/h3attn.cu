@@ -540,8 +540,9 @@ h3_status h3_varlen_attn_fwd_sage(const void *q, const void *k, const void *v, v
     qp.rope = rt;
     const dim3 qgrid(static_cast<unsigned>((max_seqlen + 127) / 128), static_cast<unsigned>(H),
                      static_cast<unsigned>(nseg));
+    const dim3 bgrid(static_cast<unsigned>((max_seqlen + 15) / 16), static_cast<unsigned>(nseg));
     h3::sage_vamax_kernel<<<qgrid, 256, 0, cs>>>(qp);
-    h3::sage_quant_kernel<<<qgrid, 256, 0, cs>>>(qp);
+    h3::sage_quant_kernel<<<bgrid, 256, 0, cs>>>(qp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
 

@@ -17,13 +17,16 @@ formulas; the reading used here (R18):
     (a block never straddles two segments); same formulas over the block.
   * V: one scale per (segment, head, channel) over the segment's tokens.
   * Scores: x = (q8 . k8) * s_q * s_k * scale * log2(e) (log2 domain).
-  * Online softmax over key tiles of 128 from the segment start, in order; the
-    running max m is updated whenever a tile raises it (the accumulator and
-    the row sum are rescaled by 2^(m_old - m_new)); P8 = e4m3(448 * 2^(x - m))
-    with m the running max including the current tile (so 448 * 2^(x - m) <=
-    448); the row sum l adds the unquantised 448 * 2^(x - m).
+  * Online softmax over key tiles of 128 from the segment start, in order,
+    with a lazily updated reference max m (log2 domain): the first tile sets
+    m to its max; a later tile raises m to the running max only when its own
+    max exceeds m by more than tau = 2 (the accumulator and the row sum are
+    then rescaled by 2^(m_old - m_new)). Hence 2^(x - m) <= 2^tau and
+    P8 = e4m3(448 * 2^-tau * 2^(x - m)) = e4m3(112 * 2^(x - m)) <= 448; the
+    row sum l adds the unquantised 112 * 2^(x - m). tau = 0 is the eager
+    update (every rise of the max rescales).
   * O = s_v * (sum_j P8_j v8_j) / l, LSE = ln(sum_j e^(scale q~.k~)) from the
-    same quantities: (m + log2(l / 448)) * ln 2.
+    same quantities: (m + log2(l / 112)) * ln 2.
 """
 
 from __future__ import annotations
@@ -36,6 +39,7 @@ from .attention import _as_f64
 from .rope import rope_ref
 
 E4M3_MAX = 448.0
+LAZY_LOG2 = 2.0
 _LOG2E = 1.0 / math.log(2.0)
 
 
@@ -131,28 +135,37 @@ def sage_quantize(q, k, v, cu_seqlens, pos=None, split=None, theta=10000.0,
 
 # ------------------------------------------------------------------- attention
 
-def _online_rows(xs, v8, kv_tile):
+def p_scale(tau: float) -> float:
+    """The P8 scale 448 * 2^-tau of the module docstring."""
+    return E4M3_MAX * 2.0 ** -tau
+
+
+def _online_rows(xs, v8, kv_tile, tau):
     """xs [R, L] scores (log2 domain), v8 [L, D] codes -> (acc [R, D], l [R], m [R])
     following the online algorithm of the module docstring."""
     R, L = xs.shape
     acc = np.zeros((R, v8.shape[1]))
     l = np.zeros(R)
     m = np.full(R, -np.inf)
+    ps = p_scale(tau)
     for j0 in range(0, L, kv_tile):
         x = xs[:, j0:j0 + kv_tile]
-        m_new = np.maximum(m, x.max(axis=1))
-        f = np.where(np.isfinite(m), np.exp2(m - m_new), 0.0)
+        tmax = x.max(axis=1)
+        first = ~np.isfinite(m)
+        raise_ = first | (tmax > m + tau)
+        m_new = np.where(first, tmax, np.where(raise_, np.maximum(m, tmax), m))
+        f = np.where(first, 0.0, np.exp2(np.where(first, 0.0, m - m_new)))
         acc *= f[:, None]
         l *= f
         m = m_new
-        p = E4M3_MAX * np.exp2(x - m[:, None])
+        p = ps * np.exp2(x - m[:, None])
         acc += e4m3_round(p) @ v8[j0:j0 + kv_tile]
         l += p.sum(axis=1)
     return acc, l, m
 
 
 def sage_attention_ref(q, k, v, cu_seqlens, scale, pos=None, split=None, theta=10000.0,
-                       pair_layout="interleaved", kv_tile=128, quant=None):
+                       pair_layout="interleaved", kv_tile=128, quant=None, tau=LAZY_LOG2):
     """Returns (O [N, H, D], LSE [H, N]) of the SAGE reading; ``quant`` may pass
     a precomputed ``sage_quantize`` result."""
     qz = quant if quant is not None else sage_quantize(q, k, v, cu_seqlens, pos, split, theta,
@@ -170,15 +183,15 @@ def sage_attention_ref(q, k, v, cu_seqlens, scale, pos=None, split=None, theta=1
         for h in range(H):
             raw = q8[a:e, h] @ k8[a:e, h].T                    # exact (e4m3 products)
             xs = raw * sq[h, a:e, None] * sk[h, None, a:e] * (scale * _LOG2E)
-            acc, l, m = _online_rows(xs, v8[a:e, h], kv_tile)
+            acc, l, m = _online_rows(xs, v8[a:e, h], kv_tile, tau)
             O[a:e, h] = acc * sv[s, h][None, :].astype(np.float64) / l[:, None]
-            LSE[h, a:e] = (m + np.log2(l / E4M3_MAX)) * math.log(2.0)
+            LSE[h, a:e] = (m + np.log2(l / p_scale(tau))) * math.log(2.0)
     return O, LSE
 
 
 def sage_attention_rows_ref(q, k, v, cu_seqlens, scale, rows, heads, pos=None, split=None,
                             theta=10000.0, pair_layout="interleaved", kv_tile=128,
-                            k_block=16):
+                            k_block=16, tau=LAZY_LOG2):
     """``sage_attention_ref`` for selected query rows and heads (any size):
     quantises only the rows' own Q and their segments' K and V for those heads."""
     cu = np.asarray(cu_seqlens, dtype=np.int64)
@@ -201,7 +214,7 @@ def sage_attention_rows_ref(q, k, v, cu_seqlens, scale, rows, heads, pos=None, s
             sq = qz["s_q"][0, r - a].astype(np.float64)
             sk = qz["s_k"][0].astype(np.float64)
             xs = (q8 @ k8.T) * sq[:, None] * sk[None, :] * (scale * _LOG2E)
-            acc, l, m = _online_rows(xs, v8, kv_tile)
+            acc, l, m = _online_rows(xs, v8, kv_tile, tau)
             O[sel, hi] = acc * qz["s_v"][0, 0][None, :].astype(np.float64) / l[:, None]
-            LSE[hi, sel] = (m + np.log2(l / E4M3_MAX)) * math.log(2.0)
+            LSE[hi, sel] = (m + np.log2(l / p_scale(tau))) * math.log(2.0)
     return O, LSE

@@ -78,7 +78,7 @@ def test_quantisation_invariants():
 
 def test_lossless_inputs_uniform_scores_give_the_segment_mean():
     # entries in {0, +-c} with c = 448 * 2^-n: every quantisation and every
-    # dequantisation scale is exact; with scale 0 every P8 is exactly 448, so
+    # dequantisation scale is exact; with scale 0 every P8 is exactly 112, so
     # O is the exact segment mean of V
     rng = np.random.default_rng(302)
     seg = [37, 200, 1]
@@ -98,64 +98,93 @@ def test_lossless_inputs_uniform_scores_give_the_segment_mean():
         np.testing.assert_allclose(LSE[:, a:e], math.log(e - a), rtol=0, atol=1e-12)
 
 
-def _direct(qz, a, e, h, scale):
-    """One-pass definition with the true row max (equal to the online result
-    whenever the first key tile holds every row's max)."""
+def _direct(qz, a, e, h, scale, tau, m=None):
+    """One-pass definition with a fixed reference max m per row (the true row
+    max unless given): equal to the online result whenever the reference max
+    never moves after the first tile."""
     q8, k8, v8 = qz["q8"][a:e, h], qz["k8"][a:e, h], qz["v8"][a:e, h]
     x = (q8 @ k8.T) * qz["s_q"][h, a:e, None].astype(np.float64) \
         * qz["s_k"][h, None, a:e].astype(np.float64) * scale / math.log(2.0)
-    p = 448.0 * np.exp2(x - x.max(axis=1, keepdims=True))
+    if m is None:
+        m = x.max(axis=1)
+    p = oracle.sage.p_scale(tau) * np.exp2(x - m[:, None])
     return (e4m3_round(p) @ v8) * qz["s_v"][0, h].astype(np.float64) / p.sum(axis=1, keepdims=True)
 
 
-def test_online_equals_direct_definition_when_the_max_never_moves():
-    # key 0 of the segment aligns with every query, so the first tile holds
-    # each row's max and the running max never changes after tile 0
-    rng = np.random.default_rng(303)
-    L, H, D = 400, 1, 64
-    q = rng.standard_normal((L, H, D)).astype(np.float32) * 0.3
+def _case(L, seed, big_key=None, big=8.0):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((L, 1, 64)).astype(np.float32) * 0.3
     q[:, :, 0] = 3.0
-    k = rng.standard_normal((L, H, D)).astype(np.float32) * 0.3
-    k[0, 0, :] = 0.0
-    k[0, 0, 0] = 8.0
-    v = rng.standard_normal((L, H, D)).astype(np.float32)
-    qb, kb, vb = (synth.f32_to_bf16_bits(t) for t in (q, k, v))
+    k = rng.standard_normal((L, 1, 64)).astype(np.float32) * 0.3
+    if big_key is not None:
+        k[big_key, 0, :] = 0.0
+        k[big_key, 0, 0] = big
+    v = rng.standard_normal((L, 1, 64)).astype(np.float32)
+    return tuple(synth.f32_to_bf16_bits(t) for t in (q, k, v))
+
+
+@pytest.mark.parametrize("tau", [0.0, 2.0])
+def test_online_equals_direct_definition_when_the_max_never_moves(tau):
+    # key 0 aligns with every query, so the first tile holds each row's max
+    L = 400
+    qb, kb, vb = _case(L, 303, big_key=0)
     cu = np.array([0, L], dtype=np.int32)
     qz = oracle.sage_quantize(qb, kb, vb, cu)
-    O, _ = oracle.sage_attention_ref(qb, kb, vb, cu, 0.125, quant=qz)
-    np.testing.assert_allclose(O[:, 0], _direct(qz, 0, L, 0, 0.125), rtol=0, atol=1e-12)
+    O, _ = oracle.sage_attention_ref(qb, kb, vb, cu, 0.125, quant=qz, tau=tau)
+    np.testing.assert_allclose(O[:, 0], _direct(qz, 0, L, 0, 0.125, tau), rtol=0, atol=1e-12)
     # and one tile only: always the direct definition
     qz1 = oracle.sage_quantize(qb[:100], kb[:100], vb[:100], np.array([0, 100]))
     O1, _ = oracle.sage_attention_ref(qb[:100], kb[:100], vb[:100], np.array([0, 100]), 0.2,
-                                      quant=qz1)
-    np.testing.assert_allclose(O1[:, 0], _direct(qz1, 0, 100, 0, 0.2), rtol=0, atol=1e-12)
+                                      quant=qz1, tau=tau)
+    np.testing.assert_allclose(O1[:, 0], _direct(qz1, 0, 100, 0, 0.2, tau), rtol=0, atol=1e-12)
+
+
+def test_a_rise_below_the_threshold_keeps_the_reference_max():
+    # the key of tile 2 scores about 1 (log2 units) above tile 0's max for
+    # every row: with tau = 2 the reference stays tile 0's max (P up to 224),
+    # which is the direct definition with m = tile 0's max
+    L = 300
+    qb, kb, vb = _case(L, 304, big_key=0, big=8.0)
+    k = oracle.bf16_bits_to_f64(kb).astype(np.float32)
+    k[290, 0, :] = 0.0
+    k[290, 0, 0] = 8.0 + 1.0 / (3.0 * 0.125 / math.log(2.0))   # +1 in log2 units
+    kb = synth.f32_to_bf16_bits(k)
+    cu = np.array([0, L], dtype=np.int32)
+    qz = oracle.sage_quantize(qb, kb, vb, cu)
+    x = (qz["q8"][:, 0] @ qz["k8"][:, 0].T) * qz["s_q"][0][:, None] * qz["s_k"][0][None, :] \
+        * 0.125 / math.log(2.0)
+    m0 = x[:, :128].max(axis=1)
+    rise = x.max(axis=1) - m0
+    assert np.all((rise > 0.5) & (rise < 1.5))
+    O, _ = oracle.sage_attention_ref(qb, kb, vb, cu, 0.125, quant=qz, tau=2.0)
+    np.testing.assert_allclose(O[:, 0], _direct(qz, 0, L, 0, 0.125, 2.0, m=m0), rtol=0, atol=1e-12)
+    # with the eager update the reference moves and the result differs
+    O0, _ = oracle.sage_attention_ref(qb, kb, vb, cu, 0.125, quant=qz, tau=0.0)
+    assert not np.allclose(O0[:, 0], O[:, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(O0[:, 0], _direct(qz, 0, L, 0, 0.125, 0.0), rtol=0, atol=0.05)
 
 
 def test_online_rescaling_matters():
-    # a late tile that raises the max: the online result differs from the
-    # direct one only by P8 rounding on the earlier tiles' grid, and both stay
-    # close to exact attention
-    rng = np.random.default_rng(304)
-    L, H, D = 300, 1, 64
-    q = rng.standard_normal((L, H, D)).astype(np.float32)
-    k = rng.standard_normal((L, H, D)).astype(np.float32)
-    k[290, 0] = q.mean(axis=0)[0] * 4
-    v = rng.standard_normal((L, H, D)).astype(np.float32)
-    qb, kb, vb = (synth.f32_to_bf16_bits(t) for t in (q, k, v))
+    # a late key scoring about 5 (log2 units) above the earlier tiles: the
+    # reference max moves; the result differs from the direct one only by P8
+    # rounding on the earlier tiles' grid
+    L = 300
+    qb, kb, vb = _case(L, 305, big_key=290, big=10.0)
     cu = np.array([0, L], dtype=np.int32)
     qz = oracle.sage_quantize(qb, kb, vb, cu)
-    O, _ = oracle.sage_attention_ref(qb, kb, vb, cu, 0.125, quant=qz)
-    Od = _direct(qz, 0, L, 0, 0.125)
-    assert not np.allclose(O[:, 0], Od, rtol=0, atol=1e-12)
-    assert np.abs(O[:, 0] - Od).max() < 0.05
+    for tau in (0.0, 2.0):
+        O, _ = oracle.sage_attention_ref(qb, kb, vb, cu, 0.125, quant=qz, tau=tau)
+        Od = _direct(qz, 0, L, 0, 0.125, tau)
+        assert not np.allclose(O[:, 0], Od, rtol=0, atol=1e-12)
+        assert np.abs(O[:, 0] - Od).max() < 0.05
 
 
 def test_single_token_segments_return_dequantised_v():
     q, k, v, pos, cu = synth.draw_random_case([1, 1, 1], 2, 64, seed=305)
     O, _ = oracle.sage_attention_ref(q, k, v, cu, 0.125, pos, (16, 24, 24))
     V = oracle.bf16_bits_to_f64(v)
-    # one key: P8 = 448, O = dequantised v (per-channel scale = |v| itself, so
-    # v maps to +-448 and back exactly)
+    # one key: P8 = 112 exactly, O = dequantised v (per-channel scale = |v|
+    # itself, so v maps to +-448 and back exactly)
     np.testing.assert_allclose(O, V, rtol=1e-6, atol=0)
 
 
