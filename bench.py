@@ -423,6 +423,81 @@ def run_skip(args, wl, rank, world, local_rank):
     return 0
 
 
+def run_sage(args, wl, rank, world, local_rank):
+    """SAGE-style FP8 variant (h3_varlen_attn_fwd_sage) on the workload's
+    seeded N(0,1) inputs and positions: dense-equivalent TFLOP/s (the dense
+    FLOPs over the time of the FP8 call, its two quantisation passes
+    included), the dense kernel on the same inputs, the distance between the
+    two outputs, and two rooflines: the FP8 tensor peak (twice the measured
+    bf16 one, the nominal ratio) and the exponential unit (16 ex2 per clock
+    per SM at the sampled SM clock; one exponential per score, three
+    quarters of them on that unit). Single process only."""
+    import torch
+
+    import audio_diffusion_transformer_h3_b200 as h3
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    q, k, v = synth.draw_qkv(wl, seed=rank_seed(wl.the_seed, rank))
+    pos, cu = h3.h3_build_positions(wl.segments)
+    N, H, D = wl.n_tokens, wl.heads, wl.head_dim
+
+    def bf(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    dq, dk, dv = bf(q), bf(k), bf(v)
+    dpos, dcu = torch.from_numpy(pos).to(dev), torch.from_numpy(cu).to(dev)
+    o_s, o_d = torch.empty_like(dq), torch.empty_like(dq)
+    ws_s = h3.sage_workspace_for(N, H, D, len(wl.seg_lens), dev)
+    ws_d = h3.workspace_for(N, H, D, len(wl.seg_lens), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    with ClockSampler(str(local_rank)) as clocks:
+        ms = timed(lambda: h3.varlen_attn_fwd_sage_t(dq, dk, dv, dcu, wl.max_seqlen, dpos,
+                                                     wl.split, wl.theta, wl.softmax_scale,
+                                                     out=o_s, workspace=ws_s, stream=stream))
+    assert h3.device_status_t(ws_s) == h3.H3_OK
+    ms_dense = timed(lambda: h3.varlen_attn_fwd_t(dq, dk, dv, dcu, wl.max_seqlen, dpos,
+                                                  wl.split, wl.theta, wl.softmax_scale,
+                                                  out=o_d, workspace=ws_d, stream=stream))
+    diff = (o_s.float() - o_d.float()).abs()
+    achieved = wl.flops() / (ms * 1e-3) / 1e12
+    peaks = measured_peaks()
+    ck = clocks.summary()
+    exps = float(sum(L * L for L in wl.seg_lens)) * H
+    xu_peak = 16 * 148 * (ck["sm_mhz"] or 1965.0) * 1e6
+    line = {"metric": "SAGE-style FP8 fused varlen joint attention fwd, dense-equivalent TFLOP/s",
+            "value": achieved, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "dtype": "e4m3 (Q, K, P, V), fp32 accumulate", "data": "synthetic (synth.draw_qkv)",
+            "config": workload_config(wl),
+            "roofline": {"bound": "tensor", "achieved": achieved,
+                         "peak": 2 * peaks["bf16_sustained"], "unit": "TFLOP/s",
+                         "frac": achieved / (2 * peaks["bf16_sustained"]),
+                         "peak_kind": "fp8 dense = 2 x measured bf16 sustained"},
+            "roofline_xu": {"achieved_ex2_per_s": 0.75 * exps / (ms * 1e-3),
+                            "peak_ex2_per_s": xu_peak,
+                            "frac": 0.75 * exps / (ms * 1e-3) / xu_peak,
+                            "note": "16 ex2/clk/SM x 148 SMs at the sampled SM clock"},
+            "dense_ms_same_inputs": ms_dense, "speedup_vs_dense": ms_dense / ms,
+            "vs_dense_kernel": {"max_abs": float(diff.max()), "mean_abs": float(diff.mean())},
+            "gpu_launches": 3 * args.steps, "clocks": ck}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_qkv(args, wl, rank, world, local_rank):
     """The QKV projection with RoPE fused into its epilogue (h3_qkv_rope_gemm)
     on the DiT's shape (hidden 5376 -> 3 x 56 heads x 128) over the tokens and
@@ -512,6 +587,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--skip-threshold", type=float, default=None,
                     help="time the skip-softmax variant on frame-group inputs instead")
+    ap.add_argument("--sage", action="store_true",
+                    help="time the SAGE-style FP8 variant instead")
     ap.add_argument("--qkv-proj", action="store_true",
                     help="time the QKV projection with the fused RoPE epilogue instead")
     args = ap.parse_args()
@@ -529,6 +606,8 @@ def main():
         return run_skip(args, wl, rank, world, local_rank)
     if args.qkv_proj:
         return run_qkv(args, wl, rank, world, local_rank)
+    if args.sage:
+        return run_sage(args, wl, rank, world, local_rank)
 
     if world > 1:
         import datetime
