@@ -56,6 +56,9 @@ _lib.h3_segment_tokens.argtypes = [_c.POINTER(h3_segment_layout)]
 _lib.h3_segment_tokens.restype = _c.c_int64
 _lib.h3_build_positions.argtypes = [_c.POINTER(h3_segment_layout), _c.c_int32, _P, _c.c_int64, _P]
 _lib.h3_build_positions.restype = _c.c_int
+_lib.h3_build_positions_at.argtypes = [_c.POINTER(h3_segment_layout), _c.c_int32, _P, _P,
+                                       _c.c_int64, _P]
+_lib.h3_build_positions_at.restype = _c.c_int
 _lib.h3_rope_apply.argtypes = [_P, _P, _P, _c.c_int64, _c.c_int32, _c.c_int32, h3_rope_cfg, _P]
 _lib.h3_rope_apply.restype = _c.c_int
 _lib.h3_workspace_size.argtypes = [_c.c_int64, _c.c_int32, _c.c_int32, _c.c_int32]
@@ -92,7 +95,7 @@ _lib.h3_status_string.restype = _c.c_char_p
 _lib.h3_last_cuda_error.argtypes = []
 _lib.h3_last_cuda_error.restype = _c.c_int32
 
-EXPORTED = ("h3_segment_tokens", "h3_build_positions", "h3_rope_apply", "h3_workspace_size",
+EXPORTED = ("h3_segment_tokens", "h3_build_positions", "h3_build_positions_at", "h3_rope_apply", "h3_workspace_size",
             "h3_varlen_attn_fwd", "h3_varlen_attn_fwd_skip", "h3_read_skip_count",
             "h3_qkv_rope_gemm", "h3_sage_workspace_size", "h3_varlen_attn_fwd_sage",
             "h3_varlen_attn_fwd_static", "h3_selftest_bounded_wait",
@@ -207,11 +210,12 @@ def h3_read_device_status(workspace: int, stream: int) -> int:
     return int(_lib.h3_read_device_status(workspace, stream))
 
 
-def h3_build_positions(layouts):
+def h3_build_positions(layouts, t_origins=None):
     """Host position build. ``layouts``: objects with the attributes of
     ``h3_segment_layout`` (or of a segment description with ``video``,
     ``audio_tail``, ``image_refs``, ``image_grid``, ``audio_refs``,
-    ``audio_ref_len``, ``audio_rate``). Returns (pos float32 [N, 3],
+    ``audio_ref_len``, ``audio_rate``); ``t_origins``: optional clock origin
+    per segment (h3_build_positions_at). Returns (pos float32 [N, 3],
     cu_seqlens int32 [nseg + 1]) as NumPy arrays."""
     import numpy as np
     segs = (h3_segment_layout * max(1, len(layouts)))()
@@ -220,8 +224,15 @@ def h3_build_positions(layouts):
     total = sum(max(0, h3_segment_tokens(segs[i])) for i in range(len(layouts)))
     pos = np.zeros((max(total, 1), 3), dtype=np.float32)
     cu = np.zeros(len(layouts) + 1, dtype=np.int32)
-    st = _lib.h3_build_positions(segs, len(layouts), pos.ctypes.data, total,
-                                 cu.ctypes.data)
+    if t_origins is None:
+        st = _lib.h3_build_positions(segs, len(layouts), pos.ctypes.data, total,
+                                     cu.ctypes.data)
+    else:
+        org = np.ascontiguousarray(t_origins, dtype=np.float64)
+        if org.shape != (len(layouts),):
+            raise ValueError("one clock origin per segment")
+        st = _lib.h3_build_positions_at(segs, len(layouts), org.ctypes.data,
+                                        pos.ctypes.data, total, cu.ctypes.data)
     _check(st, "h3_build_positions")
     return pos[:total], cu
 

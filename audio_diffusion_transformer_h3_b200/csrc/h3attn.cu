@@ -334,7 +334,16 @@ int64_t h3_segment_tokens(const h3_segment_layout *s) {
 
 h3_status h3_build_positions(const h3_segment_layout *segs, int32_t nseg, float *pos,
                              int64_t capacity, int32_t *cu_seqlens) {
+    return h3_build_positions_at(segs, nseg, nullptr, pos, capacity, cu_seqlens);
+}
+
+h3_status h3_build_positions_at(const h3_segment_layout *segs, int32_t nseg,
+                                const double *t_origin, float *pos, int64_t capacity,
+                                int32_t *cu_seqlens) {
     if (nseg < 0 || (nseg > 0 && segs == nullptr) || capacity < 0) return H3_ERR_INVALID_ARG;
+    if (t_origin != nullptr)
+        for (int32_t s = 0; s < nseg; ++s)
+            if (!std::isfinite(t_origin[s])) return H3_ERR_INVALID_ARG;
     int64_t total = 0;
     for (int32_t s = 0; s < nseg; ++s) {
         const int64_t n = h3_segment_tokens(&segs[s]);
@@ -349,7 +358,7 @@ h3_status h3_build_positions(const h3_segment_layout *segs, int32_t nseg, float 
     if (cu_seqlens) cu_seqlens[0] = 0;
     for (int32_t s = 0; s < nseg; ++s) {
         const h3_segment_layout &g = segs[s];
-        double t0 = 0.0;
+        double t0 = t_origin != nullptr ? t_origin[s] : 0.0;
         auto put = [&](double t, double h, double w) {
             pos[3 * n + 0] = static_cast<float>(t);
             pos[3 * n + 1] = static_cast<float>(h);

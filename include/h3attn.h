@@ -101,6 +101,19 @@ int64_t h3_segment_tokens(const h3_segment_layout *seg);
 h3_status h3_build_positions(const h3_segment_layout *segs, int32_t nseg, float *pos,
                              int64_t capacity, int32_t *cu_seqlens);
 
+/* h3_build_positions with a clock origin per segment: segment s starts at
+ * t0 = t_origin[s] instead of 0 (every other rule unchanged), which places a
+ * long-video continuation chunk on the global temporal RoPE clock ("MiniMax
+ * H3" vLLM-Omni recipe, section "Long video and driving audio": latent
+ * continuation with global temporal RoPE positions). The attention calls need
+ * no change: positions are their input.
+ *   t_origin: host double [nseg], finite, or NULL (all 0, h3_build_positions).
+ * Returns H3_ERR_INVALID_ARG for a non-finite origin and as h3_build_positions
+ * otherwise. Host only. */
+h3_status h3_build_positions_at(const h3_segment_layout *segs, int32_t nseg,
+                                const double *t_origin, float *pos, int64_t capacity,
+                                int32_t *cu_seqlens);
+
 /* Standalone rotary pass: out = RoPE(x, pos). "Day 0 Support for MiniMax-H3
  * on AMD Instinct GPUs", section "The diffusion transformer (DiT)".
  *   x, out : device bf16 [N, H, D], 16-byte aligned; out may equal x

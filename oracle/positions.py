@@ -20,6 +20,10 @@ Readings (the pages print no formula):
 * an audio reference of len tokens at rate r tokens per clock unit puts
   token i at t0 + i/r (h = w = 0) and advances the clock by len/r;
 * order inside a segment: image refs, audio refs, video grid, audio tail.
+* latent continuation ("MiniMax H3" vLLM-Omni recipe, section "Long video and
+  driving audio": continuation chunks use global temporal RoPE positions): a
+  segment may start its clock at an origin t_origin instead of 0; every
+  position of the segment is then formed from t0 = t_origin.
 Every value is formed in float64 with the operation order written here and
 rounded once to float32.
 """
@@ -29,15 +33,16 @@ from __future__ import annotations
 import numpy as np
 
 
-def segment_positions(layout) -> np.ndarray:
-    """Positions of one segment as float32 [L, 3] (t, h, w).
+def segment_positions(layout, t_origin: float = 0.0) -> np.ndarray:
+    """Positions of one segment as float32 [L, 3] (t, h, w), its clock
+    starting at ``t_origin``.
 
     ``layout`` has the attributes of ``synth.SegmentLayout``: video (T, Hg,
     Wg), audio_tail, image_refs, image_grid (ih, iw), audio_refs,
     audio_ref_len, audio_rate.
     """
     rows: list[tuple[float, float, float]] = []
-    t0 = 0.0
+    t0 = float(t_origin)
     ih, iw = layout.image_grid
     for _ in range(layout.image_refs):
         for h in range(ih):
@@ -62,9 +67,11 @@ def segment_positions(layout) -> np.ndarray:
     return np.asarray(rows, dtype=np.float64).astype(np.float32)
 
 
-def packed_positions(layouts) -> np.ndarray:
-    """Positions of consecutive packed segments, float32 [N, 3]."""
-    parts = [segment_positions(l) for l in layouts]
+def packed_positions(layouts, t_origins=None) -> np.ndarray:
+    """Positions of consecutive packed segments, float32 [N, 3]; segment s's
+    clock starts at t_origins[s] (0 for all when None)."""
+    origins = [0.0] * len(layouts) if t_origins is None else list(t_origins)
+    parts = [segment_positions(l, o) for l, o in zip(layouts, origins)]
     if not parts:
         return np.zeros((0, 3), dtype=np.float32)
     return np.concatenate(parts, axis=0)

@@ -117,6 +117,34 @@ def test_host_positions_edge_layouts():
     assert list(cu) == [0, 0, 1, 1 + 12 + 10 + 30 + 7, 1 + 12 + 10 + 30 + 7 + 9]
 
 
+@pytest.mark.parametrize("name", ["packed", "max"])
+def test_host_positions_with_clock_origins_match_oracle_bitwise(name):
+    # long-video continuation: each segment's clock starts at a global origin
+    wl = synth.workload(name)
+    origins = [37.25 + 1000.0 * s for s in range(len(wl.segments))]
+    pos, cu = h3.h3_build_positions(wl.segments, t_origins=origins)
+    want = oracle.packed_positions(wl.segments, origins)
+    assert np.array_equal(pos.view(np.uint32), want.view(np.uint32))
+    assert np.array_equal(cu, synth.cu_seqlens_of(wl.seg_lens))
+    zero, _ = h3.h3_build_positions(wl.segments, t_origins=[0.0] * len(wl.segments))
+    assert np.array_equal(zero.view(np.uint32),
+                          h3.h3_build_positions(wl.segments)[0].view(np.uint32))
+
+
+def test_host_positions_origin_errors():
+    seg = h3.h3_segment_layout(0, 0, 0, 0, 0, 32, 2, 2, 2, 0)
+    arr = (h3.h3_segment_layout * 1)(seg)
+    buf = np.zeros((8, 3), np.float32)
+    for bad in (float("nan"), float("inf")):
+        org = np.array([bad])
+        assert h3._lib.h3_build_positions_at(arr, 1, org.ctypes.data, buf.ctypes.data, 8,
+                                             None) == h3.H3_ERR_INVALID_ARG
+    org = np.array([5.0])
+    assert h3._lib.h3_build_positions_at(arr, 1, org.ctypes.data, buf.ctypes.data, 8,
+                                         None) == h3.H3_OK
+    assert buf[0, 0] == 5.0 and buf[4, 0] == 6.0
+
+
 def test_host_positions_errors():
     seg = h3.h3_segment_layout(0, 0, 0, 1, 4, 0, 1, 1, 1, 0)   # audio refs with rate 0
     arr = (h3.h3_segment_layout * 1)(seg)

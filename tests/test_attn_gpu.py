@@ -213,6 +213,29 @@ def test_skewed_keys_large_logits():
 
 # ------------------------------------------------------------- error paths
 
+def test_continuation_chunk_on_the_global_clock():
+    # long-video continuation: a chunk whose clock starts at latent frame 1441
+    # (positions from h3_build_positions_at); parity with the oracle, and the
+    # same attention as at origin 0 up to rounding (RoPE sees differences only)
+    h3 = _h3()
+    lay = [synth.SegmentLayout(video=(4, 12, 21), audio_tail=128),
+           synth.SegmentLayout(video=(2, 12, 21), audio_tail=64)]
+    pos0, cu = h3.h3_build_positions(lay)
+    pos1, _ = h3.h3_build_positions(lay, t_origins=[1441.0, 9.5])
+    assert np.array_equal(pos1, oracle.packed_positions(lay, [1441.0, 9.5]))
+    N = int(cu[-1])
+    rng = np.random.default_rng(41)
+    q, k, v = (synth.f32_to_bf16_bits(rng.standard_normal((N, 2, 128), dtype=np.float32))
+               for _ in range(3))
+    split, scale = (32, 48, 48), 128 ** -0.5
+    o1, l1 = _run(q, k, v, cu, 1136, pos1, split, scale)
+    O1, L1 = oracle.attention_ref(q, k, v, cu, scale, pos1, split)
+    assert_close_bf16(host_f64(o1), O1, "continuation chunk")
+    np.testing.assert_allclose(host_f64(l1), L1, rtol=0, atol=1e-2)
+    o0, _ = _run(q, k, v, cu, 1136, pos0, split, scale)
+    assert_close_bf16(host_f64(o1), host_f64(o0), "origin 1441 vs 0")
+
+
 def test_bad_cu_seqlens_sets_device_status_without_fault():
     import torch
     h3 = _h3()

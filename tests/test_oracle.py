@@ -302,6 +302,22 @@ def test_attention_invariant_to_shifting_a_segments_clock():
     assert np.abs(O3[6:] - O[6:]).max() > 1e-6
 
 
+def test_positions_clock_origin_shifts_t_only():
+    # a continuation chunk on the global clock: with an origin that keeps the
+    # values exact in float32 (integer video frames, audio steps of 1/32), every
+    # t moves by the origin and h, w stay
+    lay = synth.SegmentLayout(video=(3, 4, 5), audio_tail=96, image_refs=1,
+                              image_grid=(2, 2), audio_refs=1, audio_ref_len=64,
+                              audio_rate=32)
+    base = oracle.segment_positions(lay)
+    shifted = oracle.segment_positions(lay, 1441.0)
+    np.testing.assert_array_equal(shifted[:, 1:], base[:, 1:])
+    np.testing.assert_array_equal(shifted[:, 0].astype(np.float64),
+                                  base[:, 0].astype(np.float64) + 1441.0)
+    two = oracle.packed_positions([lay, lay], [0.0, 1441.0])
+    np.testing.assert_array_equal(two, np.concatenate([base, shifted]))
+
+
 def test_rope_inside_attention_equals_prerotated_inputs():
     q, k, v, pos, cu, split = _tiny_case([5, 4], seed=19)
     O, L = oracle.attention_ref(q, k, v, cu, 0.4, pos, split)
