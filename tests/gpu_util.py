@@ -5,7 +5,7 @@ No arithmetic of the method lives here.
 
 import numpy as np
 
-# Spec tolerance for bf16 outputs against the float64 oracle.
+# Tolerance of the path for bf16 outputs against the float64 oracle.
 MAX_ABS = 2e-2
 MEAN_ABS = 2e-3
 
