@@ -2,7 +2,6 @@
 the header declares, rejects bad arguments on the host before any CUDA call,
 and builds positions on the host bit-identically to the oracle."""
 
-import ctypes
 import os
 import re
 import subprocess

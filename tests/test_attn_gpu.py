@@ -14,7 +14,7 @@ import pytest
 
 import oracle
 import synth
-from gpu_util import MAX_ABS, MEAN_ABS, assert_close_bf16, dev, dev_bf16, host_bits, host_f64
+from gpu_util import assert_close_bf16, dev, dev_bf16, host_bits, host_f64
 
 pytestmark = pytest.mark.gpu
 
