@@ -7,7 +7,8 @@
   of a packed sequence (the shard boundary falls inside a document); the two
   all-to-alls around the attention must reproduce, on each rank's tokens,
   the attention of the whole packed sequence. The attention step is the
-  float64 oracle here, so this checks the data movement exactly.
+  float64 oracle here (dense, then the SAGE-style FP8 reading), so this
+  checks the data movement exactly.
 """
 
 import math
@@ -31,6 +32,15 @@ def _oracle_attn(q, k, v, cu, max_seqlen, pos, split, theta, scale, return_lse=F
     import oracle
     O, L = oracle.attention_ref(q.numpy(), k.numpy(), v.numpy(), cu.numpy(), scale,
                                 None if pos is None else pos.numpy(), split, theta)
+    O, L = torch.from_numpy(O), torch.from_numpy(L)
+    return (O, L) if return_lse else O
+
+
+def _sage_oracle_attn(q, k, v, cu, max_seqlen, pos, split, theta, scale, return_lse=False):
+    import torch
+    import oracle
+    O, L = oracle.sage_attention_ref(q.numpy(), k.numpy(), v.numpy(), cu.numpy(), scale,
+                                     None if pos is None else pos.numpy(), split, theta)
     O, L = torch.from_numpy(O), torch.from_numpy(L)
     return (O, L) if return_lse else O
 
@@ -76,6 +86,16 @@ def _worker(rank, world, port, root, errors):
         assert out.shape == (hi - lo, H, D) and lse.shape == (H, hi - lo)
         np.testing.assert_allclose(out.numpy(), O[lo:hi], rtol=0, atol=1e-12)
         np.testing.assert_allclose(lse.numpy(), L[:, lo:hi], rtol=0, atol=1e-12)
+        # the SAGE-style FP8 attention quantises per head (Q per token, K per 16-key
+        # block, V per segment and channel), so head sharding reproduces it exactly
+        out, lse = ulysses_attention(Q[lo:hi].contiguous(), K[lo:hi].contiguous(),
+                                     V[lo:hi].contiguous(), torch.from_numpy(cu), max(seg),
+                                     torch.from_numpy(pos), split, 1e4, scale,
+                                     attn=_sage_oracle_attn, return_lse=True)
+        Os, Ls = oracle.sage_attention_ref(Q.numpy(), K.numpy(), V.numpy(), cu, scale, pos,
+                                           split, 1e4)
+        np.testing.assert_allclose(out.numpy(), Os[lo:hi], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse.numpy(), Ls[:, lo:hi], rtol=0, atol=1e-12)
         # heads that do not split over the ranks are refused
         with pytest.raises(ValueError):
             ulysses_attention(Q[lo:hi, :3].contiguous(), K[lo:hi, :3].contiguous(),
