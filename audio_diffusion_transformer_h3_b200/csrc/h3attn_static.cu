@@ -8,16 +8,23 @@
 // uses a scratch array compiled into the library instead: a file-scope
 // __device__ array of H3_STATIC_WORKSPACE_BYTES, which the CUDA driver places
 // in device memory when it loads this file's module on a device and keeps
-// there until the process exits. Because it lives in its own translation
-// unit, the array is only loaded on devices where this entry point is used.
+// there until the process exits. Under CUDA's lazy module loading (the
+// default, CUDA_MODULE_LOADING=LAZY) the module, and with it the array, is
+// loaded only on devices where this entry point is called; with
+// CUDA_MODULE_LOADING=EAGER every context that maps the library loads it and
+// holds the array, whether or not this entry point is ever used.
 //
-// In host code `g_static_ws` names a host-side shadow, not device memory; the
-// device address is obtained once per device with cudaGetSymbolAddress (with
-// that device current) and only that address is passed to the kernels.
+// In host code `g_static_ws` names a host-side shadow, not device memory. The
+// device address is looked up with cudaGetSymbolAddress, with the calling
+// device current, on every call (once the module is loaded this is a host-side
+// table lookup), and only that address is passed to the kernels. Looking it
+// up on every call rather than caching it keeps the entry point valid when
+// the primary context is destroyed and recreated (cudaDeviceReset), which
+// reloads the module and may place the array at a new address. The first call
+// on a device loads the module, so it should come before any stream capture.
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 
 #include "h3attn.h"
 
@@ -25,24 +32,12 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_static_ws[H3_STATIC_WORKSPACE_BYTES];
 
-constexpr int kMaxDevices = 64;
-void *g_static_ptr[kMaxDevices] = {};
-std::mutex g_static_mu;
-
-// Device address of the scratch array on the current device (set-up on the
-// first call per device).
+// Device address of the scratch array on the current device.
 h3_status static_workspace(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return H3_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return H3_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_static_mu);
-    if (g_static_ptr[dev] == nullptr) {
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_static_ws) != cudaSuccess || ptr == nullptr)
-            return H3_ERR_CUDA;
-        g_static_ptr[dev] = ptr;
-    }
-    *out = g_static_ptr[dev];
+    void *ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_ws);
+    if (e != cudaSuccess || ptr == nullptr) return H3_ERR_CUDA;
+    *out = ptr;
     return H3_OK;
 }
 
@@ -54,6 +49,11 @@ extern "C" h3_status h3_varlen_attn_fwd_static(const void *q, const void *k, con
                                                const float *pos, h3_rope_cfg rope, int64_t N,
                                                int32_t H, int32_t D, float softmax_scale,
                                                h3_stream_t stream) {
+    // The shape checks of h3_varlen_attn_fwd come first, so that a call that
+    // is both malformed and too large reports the same status as there.
+    if (N < 0 || N > INT32_MAX - 1 || H < 1 || H > 65535 || nseg < 1 || nseg > 65535)
+        return H3_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return H3_ERR_UNSUPPORTED;
     // the scratch holds the status block and the rotated keys, bf16 [N, H, D];
     // every other argument is checked by h3_varlen_attn_fwd
     if (h3_workspace_size(N, H, D, nseg) > static_cast<size_t>(H3_STATIC_WORKSPACE_BYTES))

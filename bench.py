@@ -168,6 +168,21 @@ def job_tflops(world: int, flops_per_rank_step: float, steps: int, max_ms: float
 
 # ---------------------------------------------------------------- CPU oracle
 
+def host_cpu() -> dict:
+    """The machine the CPU baseline ran on: logical CPUs (os.cpu_count()) and
+    the model name that lscpu reports."""
+    model = None
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.lower().startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except Exception:
+        model = None
+    return {"host_cpu_count": os.cpu_count(), "cpu_model": model}
+
+
 def cpu_oracle_sample(wl, q, k, v, pos, cu, budget_s: float):
     """Time the float64 oracle on (head, 128-row block) units of the workload
     until ``budget_s`` seconds are spent. Returns (TFLOP/s, description, threads)."""
@@ -224,7 +239,9 @@ def run_reference(args, wl, rank, world):
             "data": "synthetic (seeded, bf16 inputs widened to float64)",
             "config": workload_config(wl), "impl": "reference",
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": desc},
+                             "sample": desc, "blas_threads": threads, **host_cpu(),
+                             "ms_per_step_covers": "the sampled units of one step only "
+                                                   "(a bounded sample, not the whole workload)"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -431,7 +448,7 @@ def run_ours(args, wl, rank, world, local_rank):
         val, desc, threads = cpu_oracle_sample(wl, host_bits(hq), host_bits(hk), host_bits(hv),
                                                opos, cu, args.cpu_seconds)
         line["cpu_baseline"] = {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                "sample": desc}
+                                "sample": desc, "blas_threads": threads, **host_cpu()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0

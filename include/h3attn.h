@@ -260,14 +260,20 @@ h3_status h3_qkv_rope_gemm(const void *x, const void *w, void *q, void *k, void 
  * that own all device memory (their own arena or a fixed budget, allocation
  * only at start-up) cannot give h3_varlen_attn_fwd a workspace; this call
  * allocates nothing and uses a scratch array compiled into the library
- * instead (H3_STATIC_WORKSPACE_BYTES of device memory on every device where
- * it is used, held until the process exits). Arguments and results are those
- * of h3_varlen_attn_fwd without the workspace pair.
- *   Limit: N*H*D*2 + 256 <= H3_STATIC_WORKSPACE_BYTES (N*H*D <= 2^25), else
- *          H3_ERR_WORKSPACE before anything is enqueued.
- *   Set-up: the first call on a device looks up the array's device address
- *          (cudaGetSymbolAddress, with that device current); make that first
- *          call before any stream capture.
+ * instead (H3_STATIC_WORKSPACE_BYTES of device memory, held until the
+ * process exits: under CUDA's default lazy module loading only on devices
+ * where this call is used; with CUDA_MODULE_LOADING=EAGER on every device
+ * whose context maps the library). Arguments and results are those of
+ * h3_varlen_attn_fwd without the workspace pair.
+ *   Check order: N, H, nseg out of range -> H3_ERR_INVALID_ARG and D not in
+ *          {64, 128} -> H3_ERR_UNSUPPORTED (as h3_varlen_attn_fwd); then
+ *          N*H*D*2 + 256 > H3_STATIC_WORKSPACE_BYTES (N*H*D > 2^25) ->
+ *          H3_ERR_WORKSPACE; then every check of h3_varlen_attn_fwd. Nothing
+ *          is enqueued on any of these errors.
+ *   Set-up: every call looks up the array's device address on the current
+ *          device (cudaGetSymbolAddress), so the call stays valid after the
+ *          context is reset. The first call on a device also loads the
+ *          array's module; make that first call before any stream capture.
  *   Sharing: every call on a device uses the same array. Calls that can run
  *          concurrently on the GPU (different streams, no ordering) race on
  *          it and must be serialised by the caller. Each call resets the

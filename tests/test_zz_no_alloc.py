@@ -90,9 +90,19 @@ def test_static_entry_matches_workspace_entry_on_two_calls(first, second):
 
 def test_static_entry_rejects_sizes_beyond_its_scratch():
     import audio_diffusion_transformer_h3_b200 as h3
-    # N*H*D = 2^25 + 128 elements does not fit; rejected before anything is enqueued
+    # N*H*D = 2^25 + 128 elements does not fit; rejected before anything is
+    # enqueued. Every pointer is NULL: if the size check ever moved behind the
+    # argument checks, the call would still fail on the host (invalid
+    # argument) instead of launching anything.
     N, H, D = (1 << 18) + 1, 1, 128
-    st = h3.h3_varlen_attn_fwd_static(0x10000, 0x20000, 0x30000, 0x40000, 0, 0x50000, 1, N,
-                                      0x60000, h3.rope_cfg((32, 48, 48), 1e4), N, H, D, 0.1, 0)
+    st = h3.h3_varlen_attn_fwd_static(0, 0, 0, 0, 0, 0, 1, N, 0,
+                                      h3.rope_cfg((32, 48, 48), 1e4), N, H, D, 0.1, 0)
     assert st == h3.H3_ERR_WORKSPACE
+    # malformed shapes report what h3_varlen_attn_fwd reports, also when too large
+    assert h3.h3_varlen_attn_fwd_static(0, 0, 0, 0, 0, 0, 1, N, 0,
+                                        h3.rope_cfg((32, 48, 48), 1e4), N, H, 256, 0.1,
+                                        0) == h3.H3_ERR_UNSUPPORTED
+    assert h3.h3_varlen_attn_fwd_static(0, 0, 0, 0, 0, 0, 0, N, 0,
+                                        h3.rope_cfg((32, 48, 48), 1e4), N, H, D, 0.1,
+                                        0) == h3.H3_ERR_INVALID_ARG
     assert h3.h3_workspace_size(1 << 18, 1, 128, 1) <= h3.H3_STATIC_WORKSPACE_BYTES
