@@ -84,6 +84,10 @@ _lib.h3_varlen_attn_fwd_sage.restype = _c.c_int
 _lib.h3_qkv_rope_gemm.argtypes = [_P, _P, _P, _P, _P, _P, h3_rope_cfg, _c.c_int64, _c.c_int32,
                                   _c.c_int32, _c.c_int32, _P, _c.c_size_t, _P]
 _lib.h3_qkv_rope_gemm.restype = _c.c_int
+_lib.h3_qkv_rope_attn_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _c.c_int32, _c.c_int32,
+                                      _P, h3_rope_cfg, _c.c_int64, _c.c_int32, _c.c_int32,
+                                      _c.c_int32, _c.c_float, _P, _c.c_size_t, _P]
+_lib.h3_qkv_rope_attn_fwd.restype = _c.c_int
 _lib.h3_read_skip_count.argtypes = [_P, _P, _c.POINTER(_c.c_uint64)]
 _lib.h3_read_skip_count.restype = _c.c_int
 _lib.h3_selftest_bounded_wait.argtypes = [_P, _c.c_size_t, _c.c_int64, _P]
@@ -97,7 +101,8 @@ _lib.h3_last_cuda_error.restype = _c.c_int32
 
 EXPORTED = ("h3_segment_tokens", "h3_build_positions", "h3_build_positions_at", "h3_rope_apply", "h3_workspace_size",
             "h3_varlen_attn_fwd", "h3_varlen_attn_fwd_skip", "h3_read_skip_count",
-            "h3_qkv_rope_gemm", "h3_sage_workspace_size", "h3_varlen_attn_fwd_sage",
+            "h3_qkv_rope_gemm", "h3_qkv_rope_attn_fwd", "h3_sage_workspace_size",
+            "h3_varlen_attn_fwd_sage",
             "h3_varlen_attn_fwd_static", "h3_selftest_bounded_wait",
             "h3_read_device_status", "h3_status_string", "h3_last_cuda_error")
 
@@ -183,6 +188,16 @@ def h3_qkv_rope_gemm(x: int, w: int, q: int, k: int, v: int, pos: int, rope: h3_
                      stream: int) -> int:
     return int(_lib.h3_qkv_rope_gemm(x, w, q, k, v, pos, rope, N, K, H, D, workspace,
                                      workspace_bytes, stream))
+
+
+def h3_qkv_rope_attn_fwd(x: int, w: int, q: int, k: int, v: int, o: int, lse: int,
+                         cu_seqlens: int, nseg: int, max_seqlen: int, pos: int,
+                         rope: h3_rope_cfg, N: int, K: int, H: int, D: int,
+                         softmax_scale: float, workspace: int, workspace_bytes: int,
+                         stream: int) -> int:
+    return int(_lib.h3_qkv_rope_attn_fwd(x, w, q, k, v, o, lse, cu_seqlens, nseg, max_seqlen,
+                                         pos, rope, N, K, H, D, softmax_scale, workspace,
+                                         workspace_bytes, stream))
 
 
 def h3_read_skip_count(workspace: int, stream: int) -> int:
@@ -356,6 +371,46 @@ def qkv_rope_gemm_t(x, w, heads: int, head_dim: int, pos=None, split=None,
                           head_dim, workspace.data_ptr(), workspace.numel(), _stream(stream))
     _check(st, "h3_qkv_rope_gemm")
     return q, k, v
+
+
+def qkv_rope_attn_fwd_t(x, w, heads: int, head_dim: int, cu_seqlens, max_seqlen: int,
+                        pos=None, split=None, theta: float = 10000.0,
+                        softmax_scale: Optional[float] = None, qkv=None, out=None,
+                        return_lse: bool = False, workspace=None, stream=None):
+    """O (and LSE [H, N] if asked) of attention over the projection x w^T,
+    through h3_qkv_rope_attn_fwd: q and k are rotated in the projection's
+    epilogue and the attention reads them as they are. ``qkv`` receives the
+    projection ([N, H, D] bf16 each; allocated if None)."""
+    import torch
+    for t, name in ((x, "x"), (w, "w")):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 2 and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA bfloat16 matrix")
+    N, K = x.shape
+    if tuple(w.shape) != (3 * heads * head_dim, K):
+        raise ValueError(f"w must be [3*H*D, K] = [{3 * heads * head_dim}, {K}]")
+    if qkv is None:
+        qkv = tuple(torch.empty((N, heads, head_dim), dtype=torch.bfloat16, device=x.device)
+                    for _ in range(3))
+    q, k, v = qkv
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        _thd(t, name)
+    if out is None:
+        out = torch.empty_like(q)
+    lse = (torch.empty((heads, N), dtype=torch.float32, device=x.device) if return_lse
+           else None)
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=x.device)
+    nseg = int(cu_seqlens.numel()) - 1
+    scale = (1.0 / math.sqrt(head_dim)) if softmax_scale is None else float(softmax_scale)
+    rope = rope_cfg(split, theta) if pos is not None else h3_rope_cfg(0, 0, 0, 0.0)
+    st = h3_qkv_rope_attn_fwd(x.data_ptr(), w.data_ptr(), q.data_ptr(), k.data_ptr(),
+                              v.data_ptr(), out.data_ptr(),
+                              lse.data_ptr() if lse is not None else 0, cu_seqlens.data_ptr(),
+                              nseg, int(max_seqlen), pos.data_ptr() if pos is not None else 0,
+                              rope, N, K, heads, head_dim, scale, workspace.data_ptr(),
+                              workspace.numel(), _stream(stream))
+    _check(st, "h3_qkv_rope_attn_fwd")
+    return (out, lse) if return_lse else out
 
 
 def sage_workspace_for(N: int, H: int, D: int, nseg: int, device=None):

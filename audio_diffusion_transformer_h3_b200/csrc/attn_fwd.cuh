@@ -22,11 +22,18 @@
 //               write P_t as bf16 into the same TMEM columns, and finally
 //               normalise O_t and store bf16 rows (and the LSE);
 //   warp 8      MMA issuer (the whole warp runs the schedule, one elected
-//               lane issues): S_t = Q_t K_j^T (A, B from shared
-//               memory) and O_t += P_t V_j (A = P from TMEM, B = V from
-//               shared memory), ordered PV0(j-1), S0(j), PV1(j-1), S1(j) so
-//               the tensor core works on one tile while the other tile's
-//               softmax runs.
+//               lane issues): S_t = Q_t K_j^T (A, B from shared memory) and
+//               O_t += P_t V_j (A = P from TMEM, B = V from shared memory).
+//               The tile of scores is computed in two 64-key halves: the
+//               half whose TMEM columns P_t(j) does not use (keys 64..127,
+//               columns 64..127) is issued as soon as the softmax has read
+//               S_t(j) into registers; the other half after PV_t(j). P_t(j)
+//               is released in two halves of 64 keys, so the first half of
+//               PV_t(j) runs while the softmax exponentiates the second.
+//               After the softmax releases the last half of P only
+//               PV (keys 64..127) and the low half of S_t(j+1) remain on the
+//               tile's dependency chain. The warp polls the barriers of both
+//               query tiles and serves whichever is ready, PV first.
 // TMEM: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D) fp32
 // columns x 128 lanes. tcgen05.mma operations issued by one thread execute in
 // order, so S_t(j) may overwrite P_t(j-1) once PV_t(j-1) has been issued.
@@ -84,13 +91,25 @@ struct AttnCfg {
     static constexpr uint32_t COL_S0 = 0, COL_S1 = 128;
     static constexpr uint32_t COL_O0 = 256, COL_O1 = 256 + D;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr int THREADS = 320;
+    static constexpr int THREADS = 384;
+    // Registers per thread: 168 at launch (384 threads, one CTA per SM);
+    // the producer warpgroup (MMA, TMA and two idle warps) drops to
+    // REGS_PRODUCER and the two softmax warpgroups rise to REGS_SOFTMAX:
+    // 2 * 128 * 224 + 128 * 56 = 384 * 168, so the raise never waits on
+    // registers the block does not hold.
+    static constexpr int REGS_LAUNCH = 168;
+    static constexpr int REGS_SOFTMAX = 224;
+    static constexpr int REGS_PRODUCER = 56;
+    static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_PRODUCER <= THREADS * REGS_LAUNCH,
+                  "register split exceeds the launch allocation");
 };
 
 // Barrier slots (uint64 each) at OFF_BAR.
+// S_t full (both halves), S_t consumed (read into registers: its columns may
+// be overwritten), first and second half of P_t written, O_t final.
 enum : int {
     B_QFULL = 0, B_QREADY = 1, B_KFULL = 2, B_KEMPTY = 4, B_VFULL = 6, B_VEMPTY = 8,
-    B_SFULL = 10, B_PFULL = 12, B_OFULL = 14, B_DRAIN = 16, B_COUNT = 17
+    B_SFULL = 10, B_SCONS = 12, B_P1 = 14, B_P2 = 16, B_OFULL = 18, B_DRAIN = 20, B_COUNT = 22
 };
 
 __device__ __forceinline__ void raise_abort(volatile int *abort, int *status) {
@@ -122,7 +141,7 @@ __global__ void __launch_bounds__(32, 1) bounded_wait_selftest_kernel(int *statu
 // running state unchanged; if all four blocks of a query tile skip, the MMA
 // warp also drops that tile's PV.
 template <int D, bool SKIP>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -168,14 +187,17 @@ __global__ void __launch_bounds__(320, 1)
         mbar_init(&bars[B_QREADY], 256);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars[B_KFULL + s], 1);
-            mbar_init(&bars[B_KEMPTY + s], 1);
+            mbar_init(&bars[B_KEMPTY + s], 2);   // one commit per query tile
             mbar_init(&bars[B_VFULL + s], 1);
-            mbar_init(&bars[B_VEMPTY + s], 1);
+            mbar_init(&bars[B_VEMPTY + s], 2);   // one commit per query tile
             mbar_init(&bars[B_SFULL + s], 1);
-            mbar_init(&bars[B_PFULL + s], 4);
+            mbar_init(&bars[B_SCONS + s], 4);    // one arrival per softmax warp
+            mbar_init(&bars[B_P1 + s], 4);
+            mbar_init(&bars[B_P2 + s], 4);
             mbar_init(&bars[B_OFULL + s], 1);
         }
         mbar_init(&bars[B_DRAIN], 1);
+        mbar_init(&bars[B_DRAIN + 1], 1);
         *abort = 0;
         for (int i = 0; i < 8; ++i) skipword[i] = 0;
         fence_mbar_init();
@@ -184,7 +206,7 @@ __global__ void __launch_bounds__(320, 1)
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp == 9 && lane == 0) {
+    if (warp == 10 && lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
@@ -194,8 +216,12 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 9) {
+    if (warp == 11) {
+        // idle warp of the producer warpgroup
+        reg_dealloc<C::REGS_PRODUCER>();
+    } else if (warp == 10) {
         // ============================ TMA producer ============================
+        reg_dealloc<C::REGS_PRODUCER>();
         // Converged warp; the elected lane issues the copies and expect_tx.
         const uint32_t leader = elect_one();
         if (leader) mbar_arrive_expect_tx(&bars[B_QFULL], 2 * C::TILE_BYTES);
@@ -241,79 +267,103 @@ __global__ void __launch_bounds__(320, 1)
                 mbar_wait(&bars[B_VFULL + (j & 1)], (j >> 1) & 1, nullptr);
         }
         __syncwarp();
-    } else if (warp == 8) {
-        // ============================ MMA issuer ==============================
-        // The whole warp runs this schedule (waits included) so that it stays
-        // converged; only the elected lane issues the MMAs and commits.
+    } else if (warp >= 8) {
+        // ============================ MMA issuers =============================
+        // Warp 8 issues every MMA of query tile 0, warp 9 every MMA of tile 1,
+        // each in its tile's order and waiting (bounded, suspending) on that
+        // tile's barriers only. The whole warp runs the schedule so that it
+        // stays converged; only the elected lane issues the MMAs and commits.
+        // tcgen05.commit tracks the MMAs of the committing thread, so each
+        // warp's commits cover its own tile; the K and V slots are released
+        // by one commit from each warp.
+        reg_dealloc<C::REGS_PRODUCER>();
+        const int t = warp - 8;
         const uint32_t leader = elect_one();
         constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t IDESC_SH = idesc_bf16_f32(128, 64, false, false);
         constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
-        const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+        const uint32_t sQ = smem_u32(smem + C::OFF_Q) + t * C::TILE_BYTES;
         const uint32_t sK = smem_u32(smem + C::OFF_K);
         const uint32_t sV = smem_u32(smem + C::OFF_V);
-        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_QREADY], 0, abort));
-        tc_fence_after();
-        for (int j = 0; ok && j <= n_kv; ++j) {
-            for (int t = 0; ok && t < 2; ++t) {
-                const uint32_t colS = t ? C::COL_S1 : C::COL_S0;
-                const uint32_t colO = t ? C::COL_O1 : C::COL_O0;
-                if (j > 0) {  // O_t += P_t(j-1) V_{j-1}
-                    const int jj = j - 1;
-                    const int vs = jj & 1;
-                    bool w = mbar_wait(&bars[B_PFULL + t], jj & 1, abort);
-                    if (w && t == 0) w = mbar_wait(&bars[B_VFULL + vs], (jj >> 1) & 1, abort);
-                    ok = __all_sync(0xffffffffu, w);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t vbase = sV + vs * C::TILE_BYTES;
-                    bool skip_pv = false;
-                    if constexpr (SKIP) {
-                        const uint32_t tag = static_cast<uint32_t>(jj + 1);
-                        skip_pv = skipword[t * 4 + 0] == tag && skipword[t * 4 + 1] == tag &&
-                                  skipword[t * 4 + 2] == tag && skipword[t * 4 + 3] == tag;
-                    }
+        const uint32_t colS = tmem + (t ? C::COL_S1 : C::COL_S0);
+        const uint32_t colO = tmem + (t ? C::COL_O1 : C::COL_O0);
+        // S_t, or its 64-key half: key rows [r0, r0 + n) of the K tile in
+        // slot ks into TMEM columns [r0, r0 + n) of S_t
+        auto issue_s = [&](int ks, int r0, int n) {
+            const uint32_t kbase = sK + ks * C::TILE_BYTES + r0 * 128;
 #pragma unroll
-                    for (int kk = 0; kk < C::BN / 16; ++kk) {
-                        if (skip_pv) break;
-                        // V tile [128 keys][D] is MN-major for B: 8 key rows at 128 B,
-                        // groups of 8 rows at SBO = 1024 B, 64-col boxes at LBO.
-                        const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::BOX_BYTES, 1024);
-                        umma_ts_w(tmem + colO, tmem + colS + kk * 8, bdesc, IDESC_O,
-                                  (jj > 0 || kk > 0) ? 1u : 0u, leader);
-                    }
-                    if (j == n_kv) umma_commit_w(&bars[B_OFULL + t], leader);
-                    if (t == 1) umma_commit_w(&bars[B_VEMPTY + vs], leader);
-                }
-                if (j < n_kv) {  // S_t = Q_t K_j^T
-                    const int ks = j & 1;
-                    if (t == 0) {
-                        ok = __all_sync(0xffffffffu,
-                                        mbar_wait(&bars[B_KFULL + ks], (j >> 1) & 1, abort));
-                        if (!ok) break;
-                        tc_fence_after();
-                    }
-                    const uint32_t qbase = sQ + t * C::TILE_BYTES;
-                    const uint32_t kbase = sK + ks * C::TILE_BYTES;
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+                umma_ss_w(colS + r0, sdesc_sw128(sQ + off, 16, 1024),
+                          sdesc_sw128(kbase + off, 16, 1024), n == 128 ? IDESC_S : IDESC_SH,
+                          kk > 0 ? 1u : 0u, leader);
+            }
+        };
+        // O_t += P_t V_j over keys [16 k0, 16 k1) of the tile
+        auto issue_pv = [&](int j, int k0, int k1) {
+            const uint32_t vbase = sV + (j & 1) * C::TILE_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-                        const uint64_t adesc = sdesc_sw128(qbase + off, 16, 1024);
-                        const uint64_t bdesc = sdesc_sw128(kbase + off, 16, 1024);
-                        umma_ss_w(tmem + colS, adesc, bdesc, IDESC_S, kk > 0 ? 1u : 0u, leader);
-                    }
-                    umma_commit_w(&bars[B_SFULL + t], leader);
-                    if (t == 1) umma_commit_w(&bars[B_KEMPTY + ks], leader);
-                }
+            for (int kk = k0; kk < k1; ++kk) {
+                // V tile [128 keys][D] is MN-major for B: 8 key rows at 128 B,
+                // groups of 8 rows at SBO = 1024 B, 64-col boxes at LBO.
+                const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::BOX_BYTES, 1024);
+                umma_ts_w(colO, colS + kk * 8, bdesc, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u,
+                          leader);
+            }
+        };
+        auto wait = [&](int bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(&bars[bar], parity, abort));
+        };
+        bool ok = wait(B_QREADY, 0) && wait(B_KFULL, 0);
+        if (ok) {
+            tc_fence_after();
+            issue_s(0, 0, 128);
+            umma_commit_w(&bars[B_SFULL + t], leader);
+            umma_commit_w(&bars[B_KEMPTY], leader);
+        }
+        for (int j = 0; ok && j < n_kv; ++j) {
+            const bool more = j + 1 < n_kv;
+            const int ks = (j + 1) & 1;
+            // keys 64..127 of the next tile into the columns P_t(j) leaves free,
+            // as soon as the softmax holds S_t(j) in registers
+            if (more) {
+                ok = wait(B_SCONS + t, j & 1) && wait(B_KFULL + ks, ((j + 1) >> 1) & 1);
+                if (!ok) break;
+                tc_fence_after();
+                issue_s(ks, 64, 64);
+            }
+            ok = wait(B_P1 + t, j & 1) && wait(B_VFULL + (j & 1), (j >> 1) & 1);
+            if (!ok) break;
+            tc_fence_after();
+            bool skip_pv = false;
+            if constexpr (SKIP) {
+                const uint32_t tag = static_cast<uint32_t>(j + 1);
+                skip_pv = skipword[t * 4 + 0] == tag && skipword[t * 4 + 1] == tag &&
+                          skipword[t * 4 + 2] == tag && skipword[t * 4 + 3] == tag;
+            }
+            if (!skip_pv) issue_pv(j, 0, C::BN / 32);
+            ok = wait(B_P2 + t, j & 1);
+            if (!ok) break;
+            tc_fence_after();
+            if (!skip_pv) issue_pv(j, C::BN / 32, C::BN / 16);
+            umma_commit_w(&bars[B_VEMPTY + (j & 1)], leader);
+            if (more) {
+                issue_s(ks, 0, 64);
+                umma_commit_w(&bars[B_SFULL + t], leader);
+                umma_commit_w(&bars[B_KEMPTY + ks], leader);
+            } else {
+                umma_commit_w(&bars[B_OFULL + t], leader);
             }
         }
         if (!ok) {
             if (leader) raise_abort(abort, p.status);
-            umma_commit_w(&bars[B_DRAIN], leader);  // completes once every issued MMA is done
-            mbar_wait(&bars[B_DRAIN], 0, nullptr);
+            umma_commit_w(&bars[B_DRAIN + t], leader);  // completes once this warp's MMAs are done
+            mbar_wait(&bars[B_DRAIN + t], 0, nullptr);
         }
         __syncwarp();
     } else {
         // ============================ softmax / epilogue ======================
+        reg_alloc<C::REGS_SOFTMAX>();
         const int t = warp >> 2;                 // query tile of this warpgroup
         const int r = tid & 127;                 // row inside the tile = TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -362,6 +412,11 @@ __global__ void __launch_bounds__(320, 1)
             tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
             tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
             tmem_wait_ld();
+            // S_t(j) is in registers: the MMA warp may now overwrite its columns
+            // 64..127 with the next tile's scores
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[B_SCONS + t]);
             const int kv_valid = seg_end - (seg_start + j * C::BN);
             if (kv_valid < C::BN) {
 #pragma unroll
@@ -405,7 +460,8 @@ __global__ void __launch_bounds__(320, 1)
                             // blocks with no row inside the segment are not counted
                             if (p.skip_count != nullptr && q0 + t * C::BM + (warp & 3) * 32 < seg_end)
                                 atomicAdd(p.skip_count, 1ull);
-                            mbar_arrive(&bars[B_PFULL + t]);
+                            mbar_arrive(&bars[B_P1 + t]);
+                            mbar_arrive(&bars[B_P2 + t]);
                         }
                         continue;
                     }
@@ -426,38 +482,42 @@ __global__ void __launch_bounds__(320, 1)
             const float nm = -m_used;
             float lq[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             uint32_t pk[64];
-            if (kv_valid < C::BN) {
-                // keys past the segment end get P = 0 exactly (also when the
-                // scale is 0, where -inf * 0 would give NaN)
+            // P for keys [64 h, 64 h + 64) into pk[32 h .. 32 h + 31]
+            auto exp_half = [&](const int h) {
+                if (kv_valid < C::BN) {
+                    // keys past the segment end get P = 0 exactly (also when the
+                    // scale is 0, where -inf * 0 would give NaN)
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const float p0 = (2 * c < kv_valid)
-                        ? ex2_approx(fmaf(__uint_as_float(s[2 * c]), sl2, nm)) : 0.0f;
-                    const float p1 = (2 * c + 1 < kv_valid)
-                        ? ex2_approx(fmaf(__uint_as_float(s[2 * c + 1]), sl2, nm)) : 0.0f;
-                    lq[c & 3] += p0 + p1;
-                    pk[c] = pack_bf16x2(p0, p1);
-                }
-            } else {
-                // H3_FMA_EXP2_PAIRS column pairs of every eight on the FMA pipe
-                // (exp2_fma), the rest on MUFU (ex2.approx)
-#pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const float x0 = fmaf(__uint_as_float(s[2 * c]), sl2, nm);
-                    const float x1 = fmaf(__uint_as_float(s[2 * c + 1]), sl2, nm);
-                    float p0, p1;
-                    if ((c & 7) >= 8 - H3_FMA_EXP2_PAIRS) {
-                        p0 = exp2_fma(x0);
-                        p1 = exp2_fma(x1);
-                    } else {
-                        p0 = ex2_approx(x0);
-                        p1 = ex2_approx(x1);
+                    for (int c = 32 * h; c < 32 * h + 32; ++c) {
+                        const float p0 = (2 * c < kv_valid)
+                            ? ex2_approx(fmaf(__uint_as_float(s[2 * c]), sl2, nm)) : 0.0f;
+                        const float p1 = (2 * c + 1 < kv_valid)
+                            ? ex2_approx(fmaf(__uint_as_float(s[2 * c + 1]), sl2, nm)) : 0.0f;
+                        lq[c & 3] += p0 + p1;
+                        pk[c] = pack_bf16x2(p0, p1);
                     }
-                    lq[c & 3] += p0 + p1;
-                    pk[c] = pack_bf16x2(p0, p1);
+                } else {
+                    // H3_FMA_EXP2_PAIRS column pairs of every eight on the FMA pipe
+                    // (exp2_fma), the rest on MUFU (ex2.approx)
+#pragma unroll
+                    for (int c = 32 * h; c < 32 * h + 32; ++c) {
+                        const float x0 = fmaf(__uint_as_float(s[2 * c]), sl2, nm);
+                        const float x1 = fmaf(__uint_as_float(s[2 * c + 1]), sl2, nm);
+                        float p0, p1;
+                        if ((c & 7) >= 8 - H3_FMA_EXP2_PAIRS) {
+                            p0 = exp2_fma(x0);
+                            p1 = exp2_fma(x1);
+                        } else {
+                            p0 = ex2_approx(x0);
+                            p1 = ex2_approx(x1);
+                        }
+                        lq[c & 3] += p0 + p1;
+                        pk[c] = pack_bf16x2(p0, p1);
+                    }
                 }
-            }
-            l += (lq[0] + lq[1]) + (lq[2] + lq[3]);
+            };
+            exp_half(0);
+            tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
             if (__any_sync(0xffffffffu, need)) {
                 // O_t holds P V up to tile j-1 (S_t(j) completing implies every
                 // earlier MMA completed); rescale it before P_t(j) is released.
@@ -471,12 +531,17 @@ __global__ void __launch_bounds__(320, 1)
                     tmem_st32(tO + c * 32, o);
                 }
             }
-            tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[B_P1 + t]);  // one arrival per warp
+            exp_half(1);
+            l += (lq[0] + lq[1]) + (lq[2] + lq[3]);
             tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_PFULL + t]);  // one arrival per warp
+            if (lane == 0) mbar_arrive(&bars[B_P2 + t]);
         }
 
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_OFULL + t], 0, abort));

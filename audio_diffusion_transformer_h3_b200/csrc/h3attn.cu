@@ -63,9 +63,20 @@ EncodeTiledFn encode_tiled() {
 struct DeviceInfo {
     bool ready = false;
     bool sm100 = false;
+    bool attn_regs_ok = false;
     int sms = 0;
     cudaError_t err = cudaSuccess;
 };
+
+template <typename Kernel>
+bool attn_regs_cover_split(Kernel kernel, int D) {
+    cudaFuncAttributes a{};
+    if (cudaFuncGetAttributes(&a, kernel) != cudaSuccess) return false;
+    const long long need = D == 128
+        ? 2LL * 128 * h3::AttnCfg<128>::REGS_SOFTMAX + 128LL * h3::AttnCfg<128>::REGS_PRODUCER
+        : 2LL * 128 * h3::AttnCfg<64>::REGS_SOFTMAX + 128LL * h3::AttnCfg<64>::REGS_PRODUCER;
+    return static_cast<long long>(a.numRegs) * h3::AttnCfg<128>::THREADS >= need;
+}
 
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -108,6 +119,14 @@ h3_status device_info(DeviceInfo **out) {
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           h3::QkvCfg::SMEM_BYTES)) != cudaSuccess)
                 return cuda_fail(e);
+            // The attention kernels move registers between warpgroups
+            // (setmaxnreg); the raise waits for registers the block holds
+            // from launch, so refuse to launch a build whose launch
+            // allocation cannot cover the split (it would never return).
+            d.attn_regs_ok = attn_regs_cover_split(h3::attn_fwd_kernel<128, false>, 128) &&
+                             attn_regs_cover_split(h3::attn_fwd_kernel<128, true>, 128) &&
+                             attn_regs_cover_split(h3::attn_fwd_kernel<64, false>, 64) &&
+                             attn_regs_cover_split(h3::attn_fwd_kernel<64, true>, 64);
         }
         d.ready = true;
     }
@@ -231,7 +250,8 @@ h3_status attn_call(const void *q, const void *k, const void *v, void *o, float 
                     const int32_t *cu_seqlens, int32_t nseg, int32_t max_seqlen,
                     const float *pos, h3_rope_cfg rope, int64_t N, int32_t H, int32_t D,
                     float softmax_scale, void *workspace, size_t workspace_bytes,
-                    h3_stream_t stream, bool skip, float skip_threshold) {
+                    h3_stream_t stream, bool skip, float skip_threshold,
+                    bool reset_status = true) {
     if (N < 0 || N > INT32_MAX - 1 || H < 1 || H > 65535 || nseg < 1 || nseg > 65535)
         return H3_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return H3_ERR_UNSUPPORTED;
@@ -246,17 +266,20 @@ h3_status attn_call(const void *q, const void *k, const void *v, void *o, float 
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
         !aligned(pos, 4) || !aligned(lse, 4) || !aligned(cu_seqlens, 4))
         return H3_ERR_MISALIGNED;
-    if (workspace == nullptr || !aligned(workspace, 256) ||
-        workspace_bytes < h3_workspace_size(N, H, D, nseg))
+    // without positions there are no rotated keys: the status block suffices
+    const size_t need = pos != nullptr ? h3_workspace_size(N, H, D, nseg) : kStatusBytes;
+    if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need)
         return H3_ERR_WORKSPACE;
 
     DeviceInfo *d = nullptr;
     h3_status st = device_info(&d);
     if (st != H3_OK) return st;
+    if (!d->attn_regs_ok) return H3_ERR_UNSUPPORTED;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     int *status = static_cast<int *>(workspace);
     // status word (and, for the skip variant, the skipped-block counter at byte 8)
-    cudaError_t e = cudaMemsetAsync(status, 0, skip ? 16 : sizeof(int), cs);
+    cudaError_t e = reset_status ? cudaMemsetAsync(status, 0, skip ? 16 : sizeof(int), cs)
+                                 : cudaSuccess;
     if (e != cudaSuccess) return cuda_fail(e);
     if (N == 0) return H3_OK;
 
@@ -486,6 +509,31 @@ h3_status h3_qkv_rope_gemm(const void *x, const void *w, void *q, void *k, void 
         h3::qkv_rope_gemm_kernel<64><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tx, tw, p);
     e = cudaGetLastError();
     return e == cudaSuccess ? H3_OK : cuda_fail(e);
+}
+
+h3_status h3_qkv_rope_attn_fwd(const void *x, const void *w, void *q, void *k, void *v,
+                               void *o, float *lse, const int32_t *cu_seqlens, int32_t nseg,
+                               int32_t max_seqlen, const float *pos, h3_rope_cfg rope,
+                               int64_t N, int32_t K, int32_t H, int32_t D, float softmax_scale,
+                               void *workspace, size_t workspace_bytes, h3_stream_t stream) {
+    // the attention's own checks first, so that nothing is launched for a
+    // call it would refuse (its pointers are the GEMM's outputs)
+    if (N < 0 || N > INT32_MAX - 1 || H < 1 || H > 65535 || nseg < 1 || nseg > 65535)
+        return H3_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return H3_ERR_UNSUPPORTED;
+    if (!std::isfinite(softmax_scale) || softmax_scale < 0.0f || cu_seqlens == nullptr)
+        return H3_ERR_INVALID_ARG;
+    if (N > 0 && (o == nullptr || max_seqlen < 1 || max_seqlen > N)) return H3_ERR_INVALID_ARG;
+    if (!aligned(o, 16) || !aligned(lse, 4) || !aligned(cu_seqlens, 4)) return H3_ERR_MISALIGNED;
+    // q, k, v = x w^T with q and k rotated in the GEMM's epilogue; this call
+    // resets the status word
+    h3_status st = h3_qkv_rope_gemm(x, w, q, k, v, pos, rope, N, K, H, D, workspace,
+                                    workspace_bytes, stream);
+    if (st != H3_OK) return st;
+    // attention on the rotated q and k (no positions: no key pass and no
+    // rotated-key workspace); the status word keeps the GEMM's first error
+    return attn_call(q, k, v, o, lse, cu_seqlens, nseg, max_seqlen, nullptr, rope, N, H, D,
+                     softmax_scale, workspace, workspace_bytes, stream, false, 0.0f, false);
 }
 
 size_t h3_sage_workspace_size(int64_t N, int32_t H, int32_t D, int32_t nseg) {

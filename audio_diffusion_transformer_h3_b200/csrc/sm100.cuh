@@ -51,6 +51,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe: true if the phase with parity `parity` of `bar` has
+// completed. Used by the MMA warp to poll several barriers in turn.
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Cycle budget of one bounded wait (about one second at B200 clocks).
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
@@ -117,6 +131,20 @@ __device__ __forceinline__ void tc_fence_before() {
 
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Per-warpgroup register budget (executed by all four warps of a
+// warpgroup): lower this warpgroup's registers per thread to N, returning
+// the rest to the block's pool, or raise them to N from that pool. The
+// raise waits until the pool holds enough, so the warpgroups' shares must
+// add up to at most the block's launch allocation.
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // One lane of the (converged) warp: returns 1 in exactly one lane, 0 in the

@@ -665,6 +665,94 @@ def run_qkv(args, wl, rank, world, local_rank):
     return 0
 
 
+def run_qkv_attend(args, wl, rank, world, local_rank):
+    """The chained product path (h3_qkv_rope_attn_fwd) on workload ``wl``:
+    the QKV projection x [N, 5376] @ w^T (the DiT's hidden size, the
+    workload's heads) with q and k rotated in its epilogue, then the
+    attention on the rotated q and k with no key pass. Reports the chain's
+    TFLOP/s (projection 2 N K 3HD plus attention 4 L^2 H D per segment) and,
+    on the same data, the projection alone, the attention alone without
+    positions, and the dense line (key rotation pass + attention with fused
+    query rotation) on unrotated q, k, v. Single process only."""
+    import torch
+
+    import audio_diffusion_transformer_h3_b200 as h3
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    K = synth.QKV_PROJECTION.hidden
+    N, H, D = wl.n_tokens, wl.heads, wl.head_dim
+    x_bits, w_bits = synth.draw_linear_case(N, K, 3 * H * D, seed=rank_seed(91, rank))
+    pos, cu = h3.h3_build_positions(wl.segments)
+
+    def bf(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    x, w = bf(x_bits), bf(w_bits)
+    del x_bits, w_bits
+    dpos, dcu = torch.from_numpy(pos).to(dev), torch.from_numpy(cu).to(dev)
+    qkv = tuple(torch.empty((N, H, D), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    raw = tuple(torch.empty((N, H, D), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    o = torch.empty((N, H, D), dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    ws_dense = h3.workspace_for(N, H, D, len(wl.seg_lens), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    def chain():
+        h3.qkv_rope_attn_fwd_t(x, w, H, D, dcu, wl.max_seqlen, dpos, wl.split, wl.theta,
+                               wl.softmax_scale, qkv=qkv, out=o, workspace=ws, stream=stream)
+
+    with ClockSampler(str(local_rank)) as clocks:
+        ms = timed(chain)
+    assert h3.device_status_t(ws) == h3.H3_OK
+    ms_proj = timed(lambda: h3.qkv_rope_gemm_t(x, w, H, D, dpos, wl.split, wl.theta, out=qkv,
+                                               workspace=ws, stream=stream))
+    ms_attn = timed(lambda: h3.varlen_attn_fwd_t(*qkv, dcu, wl.max_seqlen, None, None,
+                                                 wl.theta, wl.softmax_scale, out=o,
+                                                 workspace=ws, stream=stream))
+    h3.qkv_rope_gemm_t(x, w, H, D, None, None, out=raw, workspace=ws, stream=stream)
+    ms_dense = timed(lambda: h3.varlen_attn_fwd_t(*raw, dcu, wl.max_seqlen, dpos, wl.split,
+                                                  wl.theta, wl.softmax_scale, out=o,
+                                                  workspace=ws_dense, stream=stream))
+    assert h3.device_status_t(ws_dense) == h3.H3_OK
+    f_proj = 2.0 * N * K * 3 * H * D
+    f_attn = wl.flops()
+    peaks = measured_peaks()
+    achieved = (f_proj + f_attn) / (ms * 1e-3) / 1e12
+    line = {"metric": "QKV projection with fused RoPE epilogue chained into varlen joint "
+                      "attention fwd, TFLOP/s",
+            "value": achieved, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic (synth.draw_linear_case: x ~ N(0,1), "
+                                     "w ~ N(0,1/K); positions of the workload)",
+            "config": {**workload_config(wl), "hidden": K,
+                       "workload": f"{wl.name}: qkv projection {N}x{K} -> 3x{H}x{D}, then "
+                                   "attention"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16"],
+                         "peak_kind": f"bf16 dense, burst ({peaks['source']})"},
+            "projection_ms": ms_proj,
+            "attention_no_key_pass_ms": ms_attn,
+            "attention_no_key_pass_tflops": f_attn / (ms_attn * 1e-3) / 1e12,
+            "dense_line_ms_same_data": ms_dense,
+            "dense_line_tflops_same_data": f_attn / (ms_dense * 1e-3) / 1e12,
+            "gpu_launches": 2 * args.steps, "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -681,6 +769,8 @@ def main():
                     help="time the SAGE-style FP8 variant instead")
     ap.add_argument("--qkv-proj", action="store_true",
                     help="time the QKV projection with the fused RoPE epilogue instead")
+    ap.add_argument("--attend", action="store_true",
+                    help="with --qkv-proj: time the projection chained into the attention")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -694,6 +784,8 @@ def main():
         return run_reference(args, wl, rank, world)
     if args.skip_threshold is not None:
         return run_skip(args, wl, rank, world, local_rank)
+    if args.qkv_proj and args.attend:
+        return run_qkv_attend(args, wl, rank, world, local_rank)
     if args.qkv_proj:
         return run_qkv(args, wl, rank, world, local_rank)
     if args.sage:

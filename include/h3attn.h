@@ -148,8 +148,9 @@ size_t h3_workspace_size(int64_t N, int32_t H, int32_t D, int32_t nseg);
  *                D in {64, 128}; 1 <= nseg <= 65535.
  *   softmax_scale : finite, >= 0 (0 gives the mean of V over the segment).
  *   workspace  : device, 256-byte aligned, >= h3_workspace_size(N, H, D, nseg)
- *                bytes; owned by the caller, must not be shared by calls that
- *                run concurrently. Its status word is reset by every call.
+ *                bytes (>= 256 bytes when pos is NULL: no rotated keys are
+ *                stored); owned by the caller, must not be shared by calls
+ *                that run concurrently. Its status word is reset by every call.
  * Accumulation is fp32; P is rounded to bf16 before the PV product; O is
  * rounded to bf16. Results are deterministic run to run. Launches: one
  * rotary kernel for k (when pos is not NULL) and one attention kernel. */
@@ -249,6 +250,34 @@ h3_status h3_qkv_rope_gemm(const void *x, const void *w, void *q, void *k, void 
                            const float *pos, h3_rope_cfg rope, int64_t N, int32_t K,
                            int32_t H, int32_t D, void *workspace, size_t workspace_bytes,
                            h3_stream_t stream);
+
+/* The QKV projection with RoPE in its epilogue, chained into the attention:
+ * h3_qkv_rope_gemm(x, w -> q, k, v, rotating q and k by pos), then
+ * h3_varlen_attn_fwd on q, k, v with pos = NULL. The keys reach the attention
+ * already rotated, so no rotary pass over k runs and no rotated-key workspace
+ * is needed; each rotation happens once, in the projection's epilogue
+ * ("MiniMax-H3 Reference" Space README, section "AoTI-compiled blocks":
+ * rotary epilogues around the block's matmuls).
+ *   x, w, pos, rope, N, K, H, D : as for h3_qkv_rope_gemm (pos may be NULL:
+ *              no rotation anywhere).
+ *   q, k, v    : device bf16 [N, H, D], written by the projection and read
+ *              by the attention (the caller owns them and may read them).
+ *   o, lse, cu_seqlens, nseg, max_seqlen, softmax_scale : as for
+ *              h3_varlen_attn_fwd.
+ *   workspace  : device, 256-byte aligned, >= 256 bytes: one status word
+ *              for both launches, reset once at the start; a bounded wait
+ *              that times out in either kernel, or invalid cu_seqlens found
+ *              by the attention kernel, leaves its code there
+ *              (h3_read_device_status).
+ * Errors: the attention's argument checks run before anything is launched,
+ * then those of h3_qkv_rope_gemm; the first failing check's status is
+ * returned. Two kernel launches (projection, attention), asynchronous on
+ * `stream`; deterministic. */
+h3_status h3_qkv_rope_attn_fwd(const void *x, const void *w, void *q, void *k, void *v,
+                               void *o, float *lse, const int32_t *cu_seqlens, int32_t nseg,
+                               int32_t max_seqlen, const float *pos, h3_rope_cfg rope,
+                               int64_t N, int32_t K, int32_t H, int32_t D, float softmax_scale,
+                               void *workspace, size_t workspace_bytes, h3_stream_t stream);
 
 /* Bytes of the scratch array compiled into the library for
  * h3_varlen_attn_fwd_static: a 256-byte status block plus room for the

@@ -190,6 +190,34 @@ def test_qkv_gemm_host_argument_errors():
     assert _qkv(workspace_bytes=255) == h3.H3_ERR_WORKSPACE
 
 
+def _chain(**over):
+    a = dict(x=0x10000, w=0x20000, q=0x30000, k=0x40000, v=0x50000, o=0x58000, lse=0x5c000,
+             cu_seqlens=0x5e000, nseg=1, max_seqlen=300, pos=0x60000,
+             rope=h3.rope_cfg((32, 48, 48), 1e4), N=300, K=256, H=2, D=128,
+             softmax_scale=0.1, workspace=0x70000, workspace_bytes=256, stream=0)
+    a.update(over)
+    return h3.h3_qkv_rope_attn_fwd(**a)
+
+
+def test_chained_projection_attention_host_argument_errors():
+    # the attention's checks first (nothing launched), then the projection's
+    assert _chain(D=96) == h3.H3_ERR_UNSUPPORTED
+    assert _chain(nseg=0) == h3.H3_ERR_INVALID_ARG
+    assert _chain(max_seqlen=0) == h3.H3_ERR_INVALID_ARG
+    assert _chain(max_seqlen=301) == h3.H3_ERR_INVALID_ARG
+    assert _chain(softmax_scale=-1.0) == h3.H3_ERR_INVALID_ARG
+    assert _chain(softmax_scale=float("nan")) == h3.H3_ERR_INVALID_ARG
+    assert _chain(cu_seqlens=0) == h3.H3_ERR_INVALID_ARG
+    assert _chain(o=0) == h3.H3_ERR_INVALID_ARG
+    assert _chain(o=0x58008) == h3.H3_ERR_MISALIGNED
+    assert _chain(lse=0x5c002) == h3.H3_ERR_MISALIGNED
+    assert _chain(K=200) == h3.H3_ERR_INVALID_ARG            # projection: K % 64 != 0
+    assert _chain(H=3) == h3.H3_ERR_INVALID_ARG              # projection: HD % 256 != 0
+    assert _chain(x=0x10008) == h3.H3_ERR_MISALIGNED
+    assert _chain(workspace=0) == h3.H3_ERR_WORKSPACE
+    assert _chain(workspace_bytes=255) == h3.H3_ERR_WORKSPACE
+
+
 def test_sage_workspace_layout_and_host_errors():
     # status | q8 k8 v8 | s_q s_k | v_amax s_v, every region 256-aligned
     N, H, nseg = 1000, 3, 2

@@ -82,18 +82,20 @@ def test_no_rope_and_scale_variants():
         assert_close_bf16(host_f64(o), O, f"no rope, scale {scale}")
 
 
-def test_single_workload_sampled_all_heads():
+def test_single_workload_full_parity():
+    # every element of the single-clip workload (8,320 tokens x 24 heads x 128),
+    # the oracle spread over the host's cores
+    from oracle_pool import attention_rows_parallel
     wl = synth.workload("single")
     q, k, v = synth.draw_qkv(wl)
     pos = oracle.packed_positions(wl.segments)
     cu = synth.cu_seqlens_of(wl.seg_lens)
     o, lse = _run(q, k, v, cu, wl.max_seqlen, pos, wl.split, wl.softmax_scale)
-    rng = np.random.default_rng(1)
-    rows = np.unique(np.r_[0:130, 8000:8320, rng.integers(0, wl.n_tokens, 300)])
-    heads = list(range(wl.heads))
-    O, L = oracle.attention_rows_ref(q, k, v, cu, wl.softmax_scale, rows, heads, pos, wl.split)
-    assert_close_bf16(host_f64(o)[rows], O, "single")
-    np.testing.assert_allclose(host_f64(lse)[:, rows], L, rtol=0, atol=1e-2)
+    rows = np.arange(wl.n_tokens)
+    O, L = attention_rows_parallel(q, k, v, cu, wl.softmax_scale, rows, range(wl.heads), pos,
+                                   wl.split, wl.theta)
+    assert_close_bf16(host_f64(o), O, "single (all elements)")
+    np.testing.assert_allclose(host_f64(lse), L, rtol=0, atol=1e-2)
 
 
 # ----------------------------------------- full-size workloads, sampled rows
@@ -107,6 +109,30 @@ def _sample_rows(cu, rng, per_seg=48):
         rows += [r for r in cand if a <= r < e]
         rows += list(rng.integers(a, e, per_seg))
     return np.unique(np.asarray(rows, dtype=np.int64))
+
+
+@pytest.mark.parametrize("name", ["long", "packed", "max"])
+def test_large_workloads_complete_heads(name):
+    # two complete heads (every query row of every segment) of the full-size
+    # workload, in the launch configuration the benchmark times: head 0 and
+    # a seeded other head; the oracle spread over the host's cores
+    import torch
+    from oracle_pool import attention_rows_parallel
+    wl = synth.workload(name)
+    q, k, v = synth.draw_qkv(wl)
+    pos = oracle.packed_positions(wl.segments)
+    cu = synth.cu_seqlens_of(wl.seg_lens)
+    o, lse = _run(q, k, v, cu, wl.max_seqlen, pos, wl.split, wl.softmax_scale)
+    heads = [0, int(np.random.default_rng(wl.index + 100).integers(1, wl.heads))]
+    got = host_f64(o[:, heads])
+    got_lse = host_f64(lse[heads])
+    del o, lse
+    torch.cuda.empty_cache()
+    rows = np.arange(wl.n_tokens)
+    O, L = attention_rows_parallel(q, k, v, cu, wl.softmax_scale, rows, heads, pos, wl.split,
+                                   wl.theta)
+    assert_close_bf16(got, O, f"{name} heads {heads} (every row)")
+    np.testing.assert_allclose(got_lse, L, rtol=0, atol=1e-2)
 
 
 @pytest.mark.parametrize("name", ["long", "packed", "max"])

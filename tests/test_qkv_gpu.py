@@ -161,3 +161,53 @@ def test_dit_projection_full_size_sampled():
     _check(q[idx], Q, "q")
     _check(k[idx], Kr, "k")
     _check(v[idx], V, "v")
+
+
+# ------------------------------------------ projection chained into attention
+
+def test_chained_projection_attention_single_workload_in_full():
+    # h3_qkv_rope_attn_fwd on the single-clip workload (8,320 tokens, 24 heads,
+    # hidden 5,376 as in the DiT): the projection rotates q and k in its
+    # epilogue and the attention reads them without positions. Every output
+    # element is compared with the float64 oracle chain (projection, rotation,
+    # attention, no intermediate rounding) within the path's tolerance.
+    import torch
+    from oracle_pool import attention_rows_parallel
+    h3 = _h3()
+    wl = synth.workload("single")
+    H, D, K = wl.heads, wl.head_dim, synth.QKV_PROJECTION.hidden
+    x, w = synth.draw_linear_case(wl.n_tokens, K, 3 * H * D, seed=141)
+    pos, cu = h3.h3_build_positions(wl.segments)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    qkv = tuple(torch.empty((wl.n_tokens, H, D), dtype=torch.bfloat16, device="cuda")
+                for _ in range(3))
+    o, lse = h3.qkv_rope_attn_fwd_t(dev_bf16(x), dev_bf16(w), H, D, dev(cu), wl.max_seqlen,
+                                    dev(pos), wl.split, wl.theta, wl.softmax_scale, qkv=qkv,
+                                    return_lse=True, workspace=ws)
+    torch.cuda.synchronize()
+    assert h3.device_status_t(ws) == h3.H3_OK
+    Q, Kr, V = oracle.qkv_rope_ref(x, w, H, D, oracle.packed_positions(wl.segments), wl.split,
+                                   wl.theta)
+    for got, want, name in ((qkv[0], Q, "q"), (qkv[1], Kr, "k"), (qkv[2], V, "v")):
+        _check(got, want, f"chained projection {name}")
+    O, L = attention_rows_parallel(Q, Kr, V, cu, wl.softmax_scale, np.arange(wl.n_tokens),
+                                   range(H))
+    assert_close_bf16(host_f64(o), O, "chained projection + attention (all elements)")
+    np.testing.assert_allclose(host_f64(lse), L, rtol=0, atol=1e-2)
+
+
+def test_chained_projection_attention_equals_the_two_calls_bitwise():
+    # the chain is the projection followed by the attention without positions
+    import torch
+    h3 = _h3()
+    seg = [300, 129, 1000]
+    N, K, H, D, split = sum(seg), 256, 2, 128, (32, 48, 48)
+    x, w = synth.draw_linear_case(N, K, 3 * H * D, seed=142)
+    pos = _pos(N, 143)
+    cu = synth.cu_seqlens_of(seg)
+    o1 = h3.qkv_rope_attn_fwd_t(dev_bf16(x), dev_bf16(w), H, D, dev(cu), 1000, dev(pos), split,
+                                1e4, 0.09)
+    q, k, v = _run(x, w, H, D, pos, split)
+    o2 = h3.varlen_attn_fwd_t(q, k, v, dev(cu), 1000, None, None, 1e4, 0.09)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bits(o1), host_bits(o2))
