@@ -9,31 +9,39 @@
 //   cu_seqlens).
 //
 // One CTA computes two 128-row query tiles (Q0, Q1) of one (segment, head)
-// against every 128-row key/value tile of the segment:
-//   warp 9      TMA producer (converged warp, elected lane issues): Q0/Q1
-//               once, then K_j and V_j through a
-//               two-stage ring (128B-swizzled boxes of 128 rows x 64 cols);
+// against every 128-row key/value tile of the segment. 384 threads in three
+// warpgroups:
 //   warps 0-7   softmax, one thread per query row (warpgroup t owns Q_t and
 //               TMEM lanes 0..127): rotate their Q row in shared memory
 //               (RoPE fused into the Q tile load), then per KV tile read S_t
 //               from TMEM, mask keys past the segment end, keep a running
 //               row max m and sum l (online softmax in the log2 domain, the
 //               O rescale skipped unless the max grows by more than 2^8),
-//               write P_t as bf16 into the same TMEM columns, and finally
-//               normalise O_t and store bf16 rows (and the LSE);
-//   warp 8      MMA issuer (the whole warp runs the schedule, one elected
-//               lane issues): S_t = Q_t K_j^T (A, B from shared memory) and
-//               O_t += P_t V_j (A = P from TMEM, B = V from shared memory).
-//               The tile of scores is computed in two 64-key halves: the
-//               half whose TMEM columns P_t(j) does not use (keys 64..127,
-//               columns 64..127) is issued as soon as the softmax has read
-//               S_t(j) into registers; the other half after PV_t(j). P_t(j)
-//               is released in two halves of 64 keys, so the first half of
-//               PV_t(j) runs while the softmax exponentiates the second.
-//               After the softmax releases the last half of P only
-//               PV (keys 64..127) and the low half of S_t(j+1) remain on the
-//               tile's dependency chain. The warp polls the barriers of both
-//               query tiles and serves whichever is ready, PV first.
+//               write P_t as bf16 into the first 64 TMEM columns of S_t in
+//               two halves of 64 keys, and finally normalise O_t and store
+//               bf16 rows (and the LSE). Warps w and w + 4 share an SM
+//               sub-partition; they take turns on its exponential unit (tile
+//               0 exponentiates key tile j, then tile 1 key tile j, then tile
+//               0 key tile j + 1, ...), which keeps the two tiles half a
+//               period apart so that one tile's products run while the other
+//               exponentiates. A quarter of the exponentials run as a cubic
+//               on the FMA pipe.
+//   warps 8, 9  MMA issuers, warp 8 + t for query tile t (the whole warp
+//               runs the schedule, one elected lane issues): S_t = Q_t K_j^T
+//               (A, B from shared memory) and O_t += P_t V_j (A = P from
+//               TMEM, B = V from shared memory). The score tile is computed
+//               in two 64-key halves: the half whose TMEM columns P_t(j) does
+//               not use (keys 64..127) is issued as soon as the softmax has
+//               read S_t(j) into registers, the other half after PV_t(j);
+//               PV_t(j) runs in two halves as the halves of P_t(j) arrive,
+//               so after the softmax releases the last half only PV over keys
+//               64..127 and the low half of S_t(j+1) remain on the tile's
+//               dependency chain.
+//   warp 10     TMA producer (converged warp, elected lane issues): Q0/Q1
+//               once, then K_j and V_j through a two-stage ring
+//               (128B-swizzled boxes of 128 rows x 64 cols); warp 11 idles.
+// The producer warpgroup gives up registers (setmaxnreg) to the two softmax
+// warpgroups.
 // TMEM: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D) fp32
 // columns x 128 lanes. tcgen05.mma operations issued by one thread execute in
 // order, so S_t(j) may overwrite P_t(j-1) once PV_t(j-1) has been issued.
@@ -48,13 +56,12 @@
 #include "rope.cuh"
 #include "sm100.cuh"
 
-// Column pairs out of every eight whose exponentials run on the FMA pipe
-// (exp2_fma) instead of MUFU, and whether the row max uses 3-input max.
+// Key pairs out of every eight whose exponentials run on the FMA pipe
+// (exp2_fma2, a cubic on the FMA and integer pipes) instead of MUFU: a
+// quarter of them, which shortens each softmax warp's exponential phase
+// (measured: 2 of 8 ahead of 0 and 1 of 8, level with 3 of 8).
 #ifndef H3_FMA_EXP2_PAIRS
-#define H3_FMA_EXP2_PAIRS 0
-#endif
-#ifndef H3_MAX3
-#define H3_MAX3 0
+#define H3_FMA_EXP2_PAIRS 2
 #endif
 
 namespace h3 {
@@ -87,7 +94,7 @@ struct AttnCfg {
     static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
     static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
-    static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
+    static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;  // barriers + alignment slack
     static constexpr uint32_t COL_S0 = 0, COL_S1 = 128;
     static constexpr uint32_t COL_O0 = 256, COL_O1 = 256 + D;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -109,7 +116,8 @@ struct AttnCfg {
 // be overwritten), first and second half of P_t written, O_t final.
 enum : int {
     B_QFULL = 0, B_QREADY = 1, B_KFULL = 2, B_KEMPTY = 4, B_VFULL = 6, B_VEMPTY = 8,
-    B_SFULL = 10, B_SCONS = 12, B_P1 = 14, B_P2 = 16, B_OFULL = 18, B_DRAIN = 20, B_COUNT = 22
+    B_SFULL = 10, B_SCONS = 12, B_P1 = 14, B_P2 = 16, B_OFULL = 18, B_DRAIN = 20, B_TURN = 22,
+    B_COUNT = 30
 };
 
 __device__ __forceinline__ void raise_abort(volatile int *abort, int *status) {
@@ -198,6 +206,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbar_init(&bars[B_DRAIN], 1);
         mbar_init(&bars[B_DRAIN + 1], 1);
+        for (int i = 0; i < 8; ++i) mbar_init(&bars[B_TURN + i], 1);
         *abort = 0;
         for (int i = 0; i < 8; ++i) skipword[i] = 0;
         fence_mbar_init();
@@ -289,26 +298,27 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t colO = tmem + (t ? C::COL_O1 : C::COL_O0);
         // S_t, or its 64-key half: key rows [r0, r0 + n) of the K tile in
         // slot ks into TMEM columns [r0, r0 + n) of S_t
+        const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);
+        const uint64_t dK = sdesc_sw128(sK, 16, 1024);
+        const uint64_t dV = sdesc_sw128(sV, C::BOX_BYTES, 1024);
         auto issue_s = [&](int ks, int r0, int n) {
-            const uint32_t kbase = sK + ks * C::TILE_BYTES + r0 * 128;
+            const uint64_t dk = dK + static_cast<uint64_t>((ks * C::TILE_BYTES + r0 * 128) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-                umma_ss_w(colS + r0, sdesc_sw128(sQ + off, 16, 1024),
-                          sdesc_sw128(kbase + off, 16, 1024), n == 128 ? IDESC_S : IDESC_SH,
+                const uint32_t off = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+                umma_ss_w(colS + r0, dQ + off, dk + off, n == 128 ? IDESC_S : IDESC_SH,
                           kk > 0 ? 1u : 0u, leader);
             }
         };
         // O_t += P_t V_j over keys [16 k0, 16 k1) of the tile
         auto issue_pv = [&](int j, int k0, int k1) {
-            const uint32_t vbase = sV + (j & 1) * C::TILE_BYTES;
+            const uint64_t dv = dV + static_cast<uint64_t>(((j & 1) * C::TILE_BYTES) >> 4);
 #pragma unroll
             for (int kk = k0; kk < k1; ++kk) {
                 // V tile [128 keys][D] is MN-major for B: 8 key rows at 128 B,
                 // groups of 8 rows at SBO = 1024 B, 64-col boxes at LBO.
-                const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::BOX_BYTES, 1024);
-                umma_ts_w(colO, colS + kk * 8, bdesc, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u,
-                          leader);
+                umma_ts_w(colO, colS + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4),
+                          IDESC_O, (j > 0 || kk > 0) ? 1u : 0u, leader);
             }
         };
         auto wait = [&](int bar, uint32_t parity) {
@@ -399,6 +409,21 @@ __global__ void __launch_bounds__(384, 1)
         fence_proxy_async_smem();
         mbar_arrive(&bars[B_QREADY]);
 
+        // The two query tiles take turns on the exponential unit of each SM
+        // sub-partition: warp w of tile 1 exponentiates tile j after warp w of
+        // tile 0 has finished tile j, and warp w of tile 0 exponentiates tile
+        // j + 1 after warp w of tile 1 has finished tile j (warps w and w + 4
+        // share a sub-partition).
+        auto take_turn = [&](int j) -> bool {
+            if (t == 0 && j == 0) return true;
+            const int bar = t == 0 ? B_TURN + (warp & 3) : B_TURN + 4 + (warp & 3);
+            const uint32_t par = t == 0 ? static_cast<uint32_t>((j - 1) & 1) : static_cast<uint32_t>(j & 1);
+            return __all_sync(0xffffffffu, mbar_wait(&bars[bar], par, abort));
+        };
+        auto give_turn = [&]() {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[t == 0 ? B_TURN + 4 + (warp & 3) : B_TURN + (warp & 3)]);
+        };
         float m_used = -INFINITY, l = 0.f;
         float m_run = -INFINITY;  // true running row max (skip-softmax decision)
         const float sl2 = p.scale_log2;
@@ -427,16 +452,8 @@ __global__ void __launch_bounds__(384, 1)
             float mq[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) mq[i] = __uint_as_float(s[i]);
-#if H3_MAX3
-#pragma unroll
-            for (int c = 8; c < 128; c += 16)
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    mq[i] = fmax3(mq[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 8 + i]));
-#else
 #pragma unroll
             for (int c = 8; c < 128; ++c) mq[c & 7] = fmaxf(mq[c & 7], __uint_as_float(s[c]));
-#endif
             const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
                                    fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
             const float m_new = mx * sl2;
@@ -455,6 +472,8 @@ __global__ void __launch_bounds__(384, 1)
                         tmem_wait_st();
                         tc_fence_before();
                         __syncwarp();
+                        if (!take_turn(j)) { ok = false; break; }
+                        give_turn();
                         if (lane == 0) {
                             skipword[t * 4 + (warp & 3)] = static_cast<uint32_t>(j + 1);
                             // blocks with no row inside the segment are not counted
@@ -499,23 +518,28 @@ __global__ void __launch_bounds__(384, 1)
                 } else {
                     // H3_FMA_EXP2_PAIRS column pairs of every eight on the FMA pipe
                     // (exp2_fma), the rest on MUFU (ex2.approx)
+                    const uint64_t s2 = f2_splat(sl2), n2 = f2_splat(nm);
+                    uint64_t acc0 = 0, acc1 = 0;
 #pragma unroll
                     for (int c = 32 * h; c < 32 * h + 32; ++c) {
-                        const float x0 = fmaf(__uint_as_float(s[2 * c]), sl2, nm);
-                        const float x1 = fmaf(__uint_as_float(s[2 * c + 1]), sl2, nm);
+                        float x0, x1;
+                        ffma2(x0, x1, __uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1]),
+                              s2, n2);
                         float p0, p1;
                         if ((c & 7) >= 8 - H3_FMA_EXP2_PAIRS) {
-                            p0 = exp2_fma(x0);
-                            p1 = exp2_fma(x1);
+                            exp2_fma2(p0, p1, x0, x1);
                         } else {
                             p0 = ex2_approx(x0);
                             p1 = ex2_approx(x1);
                         }
-                        lq[c & 3] += p0 + p1;
+                        if (c & 1) fadd2(acc1, p0, p1); else fadd2(acc0, p0, p1);
                         pk[c] = pack_bf16x2(p0, p1);
                     }
+                    lq[0] += f2_sum(acc0);
+                    lq[1] += f2_sum(acc1);
                 }
             };
+            if (!take_turn(j)) { ok = false; break; }
             exp_half(0);
             tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
             if (__any_sync(0xffffffffu, need)) {
@@ -536,6 +560,7 @@ __global__ void __launch_bounds__(384, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_P1 + t]);  // one arrival per warp
             exp_half(1);
+            give_turn();
             l += (lq[0] + lq[1]) + (lq[2] + lq[3]);
             tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             tmem_wait_st();

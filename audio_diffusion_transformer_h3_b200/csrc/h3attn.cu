@@ -72,10 +72,13 @@ template <typename Kernel>
 bool attn_regs_cover_split(Kernel kernel, int D) {
     cudaFuncAttributes a{};
     if (cudaFuncGetAttributes(&a, kernel) != cudaSuccess) return false;
+    using C128 = h3::AttnCfg<128>;
+    using C64 = h3::AttnCfg<64>;
     const long long need = D == 128
-        ? 2LL * 128 * h3::AttnCfg<128>::REGS_SOFTMAX + 128LL * h3::AttnCfg<128>::REGS_PRODUCER
-        : 2LL * 128 * h3::AttnCfg<64>::REGS_SOFTMAX + 128LL * h3::AttnCfg<64>::REGS_PRODUCER;
-    return static_cast<long long>(a.numRegs) * h3::AttnCfg<128>::THREADS >= need;
+        ? (C128::THREADS - 128LL) * C128::REGS_SOFTMAX + 128LL * C128::REGS_PRODUCER
+        : (C64::THREADS - 128LL) * C64::REGS_SOFTMAX + 128LL * C64::REGS_PRODUCER;
+    const int threads = D == 128 ? C128::THREADS : C64::THREADS;
+    return static_cast<long long>(a.numRegs) * threads >= need;
 }
 
 constexpr int kMaxDevices = 64;

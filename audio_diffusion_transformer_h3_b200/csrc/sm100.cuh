@@ -265,6 +265,27 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// 32 lanes x 16 consecutive 32-bit columns (as tmem_ld32, half the width).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
 // ----------------------------------------------------------------- descriptors
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
@@ -330,6 +351,67 @@ __device__ __forceinline__ float exp2_fma(float x) {
     p = __fmaf_rn(p, f, c0);
     // low bits of t hold j: bits(t) * 2^23 == j << 23 modulo 2^32
     return __uint_as_float(__float_as_uint(t) * 8388608u + __float_as_uint(p));
+}
+
+
+// ---- packed f32x2 arithmetic (sm_100: one instruction for two fp32 lanes)
+__device__ __forceinline__ uint64_t f2_splat(float a) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(a));
+    return r;
+}
+// (y0, y1) = (x0, x1) * s + c, lane-wise, s and c packed pairs
+__device__ __forceinline__ void ffma2(float &y0, float &y1, float x0, float x1, uint64_t s,
+                                      uint64_t c) {
+    asm("{\n\t.reg .b64 xa, da;\n\t"
+        "mov.b64 xa, {%2, %3};\n\t"
+        "fma.rn.f32x2 da, xa, %4, %5;\n\t"
+        "mov.b64 {%0, %1}, da;\n\t}"
+        : "=f"(y0), "=f"(y1) : "f"(x0), "f"(x1), "l"(s), "l"(c));
+}
+// acc += (a0, a1), lane-wise
+__device__ __forceinline__ void fadd2(uint64_t &acc, float a0, float a1) {
+    asm("{\n\t.reg .b64 xa;\n\t"
+        "mov.b64 xa, {%1, %2};\n\t"
+        "add.rn.f32x2 %0, %0, xa;\n\t}"
+        : "+l"(acc) : "f"(a0), "f"(a1));
+}
+__device__ __forceinline__ float f2_sum(uint64_t a) {
+    float x, y;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(a));
+    return x + y;
+}
+
+
+// 2^x for two lanes on the FMA and integer pipes (the method of exp2_fma,
+// with packed fp32 arithmetic)
+__device__ __forceinline__ void exp2_fma2(float &y0, float &y1, float x0, float x1) {
+    x0 = fmaxf(x0, -126.0f);
+    x1 = fmaxf(x1, -126.0f);
+    uint32_t t0, t1, p0, p1;
+    asm("{\n\t.reg .b64 xa, ta, ra, fa, pa, sh, nsh, nm1, c0, c1, c2, c3;\n\t"
+        "mov.b64 xa, {%4, %5};\n\t"
+        "mov.b64 sh, {%6, %6};\n\t"
+        "mov.b64 nsh, {%7, %7};\n\t"
+        "mov.b64 nm1, {%8, %8};\n\t"
+        "mov.b64 c0, {%9, %9};\n\t"
+        "mov.b64 c1, {%10, %10};\n\t"
+        "mov.b64 c2, {%11, %11};\n\t"
+        "mov.b64 c3, {%12, %12};\n\t"
+        "add.rn.f32x2 ta, xa, sh;\n\t"
+        "add.rn.f32x2 ra, ta, nsh;\n\t"
+        "fma.rn.f32x2 fa, ra, nm1, xa;\n\t"
+        "fma.rn.f32x2 pa, c3, fa, c2;\n\t"
+        "fma.rn.f32x2 pa, pa, fa, c1;\n\t"
+        "fma.rn.f32x2 pa, pa, fa, c0;\n\t"
+        "mov.b64 {%0, %1}, ta;\n\t"
+        "mov.b64 {%2, %3}, pa;\n\t}"
+        : "=r"(t0), "=r"(t1), "=r"(p0), "=r"(p1)
+        : "f"(x0), "f"(x1), "f"(12582912.0f), "f"(-12582912.0f), "f"(-1.0f),
+          "f"(0.9999284744262695f), "f"(0.6932608485221863f), "f"(0.24260516464710236f),
+          "f"(0.05516925826668739f));
+    y0 = __uint_as_float(t0 * 8388608u + p0);
+    y1 = __uint_as_float(t1 * 8388608u + p1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -319,100 +319,105 @@ def run_ours(args, wl, rank, world, local_rank):
     mean_step_ms = float(np.mean(step_ms))
 
     # ---- end-to-end through the public API with host buffers ----
-    # Every step copies its inputs from pinned host memory and reads its
-    # result back. Serial: copy in, compute, copy out on one stream. Pipelined
-    # (the reported e2e): two device slots; step i+1's inputs go up on an H2D
-    # stream and step i-1's output comes down on a D2H stream while step i's
-    # kernels run, with events ordering slot reuse.
-    h2d = hq.numel() * 2 * 3 + hpos.numel() * 4 + hcu.numel() * 4
-    d2h = ho.numel() * 2
+    # (skipped with --no-e2e, which profiling runs use to keep device memory low)
+    def run_e2e():
+        # Every step copies its inputs from pinned host memory and reads its
+        # result back. Serial: copy in, compute, copy out on one stream. Pipelined
+        # (the reported e2e): two device slots; step i+1's inputs go up on an H2D
+        # stream and step i-1's output comes down on a D2H stream while step i's
+        # kernels run, with events ordering slot reuse.
+        h2d = hq.numel() * 2 * 3 + hpos.numel() * 4 + hcu.numel() * 4
+        d2h = ho.numel() * 2
 
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        dpos.copy_(hpos, non_blocking=True)
-        dcu.copy_(hcu, non_blocking=True)
-        h3.varlen_attn_fwd_t(dq, dk, dv, dcu, wl.max_seqlen, dpos, wl.split, wl.theta,
-                             wl.softmax_scale, out=do, workspace=ws, stream=stream)
-        ho.copy_(do, non_blocking=True)
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dpos.copy_(hpos, non_blocking=True)
+            dcu.copy_(hcu, non_blocking=True)
+            h3.varlen_attn_fwd_t(dq, dk, dv, dcu, wl.max_seqlen, dpos, wl.split, wl.theta,
+                                 wl.softmax_scale, out=do, workspace=ws, stream=stream)
+            ho.copy_(do, non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
         e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_serial_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_serial_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
 
-    slots = [dict(q=dq, k=dk, v=dv, pos=dpos, cu=dcu, o=do, ws=ws, ho=ho),
-             dict(q=torch.empty_like(dq), k=torch.empty_like(dk), v=torch.empty_like(dv),
-                  pos=torch.empty_like(dpos), cu=torch.empty_like(dcu), o=torch.empty_like(do),
-                  ws=h3.workspace_for(N, H, D, nseg, dev), ho=torch.empty_like(ho).pin_memory())]
-    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        slots = [dict(q=dq, k=dk, v=dv, pos=dpos, cu=dcu, o=do, ws=ws, ho=ho),
+                 dict(q=torch.empty_like(dq), k=torch.empty_like(dk), v=torch.empty_like(dv),
+                      pos=torch.empty_like(dpos), cu=torch.empty_like(dcu), o=torch.empty_like(do),
+                      ws=h3.workspace_for(N, H, D, nseg, dev), ho=torch.empty_like(ho).pin_memory())]
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def pipelined(n_steps, start_event):
-        ev_in = [torch.cuda.Event() for _ in range(2)]
-        ev_done = [None, None]      # step's kernels done (inputs and o free to reuse)
-        ev_out = [None, None]       # step's output read back
-        up.wait_event(start_event)
+        def pipelined(n_steps, start_event):
+            ev_in = [torch.cuda.Event() for _ in range(2)]
+            ev_done = [None, None]      # step's kernels done (inputs and o free to reuse)
+            ev_out = [None, None]       # step's output read back
+            up.wait_event(start_event)
 
-        def upload(i):
-            sl = slots[i & 1]
-            with torch.cuda.stream(up):
-                if ev_done[i & 1] is not None:
-                    up.wait_event(ev_done[i & 1])
-                sl["q"].copy_(hq, non_blocking=True)
-                sl["k"].copy_(hk, non_blocking=True)
-                sl["v"].copy_(hv, non_blocking=True)
-                sl["pos"].copy_(hpos, non_blocking=True)
-                sl["cu"].copy_(hcu, non_blocking=True)
-                ev_in[i & 1].record(up)
+            def upload(i):
+                sl = slots[i & 1]
+                with torch.cuda.stream(up):
+                    if ev_done[i & 1] is not None:
+                        up.wait_event(ev_done[i & 1])
+                    sl["q"].copy_(hq, non_blocking=True)
+                    sl["k"].copy_(hk, non_blocking=True)
+                    sl["v"].copy_(hv, non_blocking=True)
+                    sl["pos"].copy_(hpos, non_blocking=True)
+                    sl["cu"].copy_(hcu, non_blocking=True)
+                    ev_in[i & 1].record(up)
 
-        upload(0)
-        for i in range(n_steps):
-            sl = slots[i & 1]
-            stream.wait_event(ev_in[i & 1])
-            if ev_out[i & 1] is not None:
-                stream.wait_event(ev_out[i & 1])
-            h3.varlen_attn_fwd_t(sl["q"], sl["k"], sl["v"], sl["cu"], wl.max_seqlen, sl["pos"],
-                                 wl.split, wl.theta, wl.softmax_scale, out=sl["o"],
-                                 workspace=sl["ws"], stream=stream)
-            done = torch.cuda.Event()
-            done.record(stream)
-            ev_done[i & 1] = done
-            if i + 1 < n_steps:
-                upload(i + 1)
-            with torch.cuda.stream(down):
-                down.wait_event(done)
-                sl["ho"].copy_(sl["o"], non_blocking=True)
-                out = torch.cuda.Event()
-                out.record(down)
-                ev_out[i & 1] = out
-        stream.wait_stream(down)
-        stream.wait_stream(up)
+            upload(0)
+            for i in range(n_steps):
+                sl = slots[i & 1]
+                stream.wait_event(ev_in[i & 1])
+                if ev_out[i & 1] is not None:
+                    stream.wait_event(ev_out[i & 1])
+                h3.varlen_attn_fwd_t(sl["q"], sl["k"], sl["v"], sl["cu"], wl.max_seqlen, sl["pos"],
+                                     wl.split, wl.theta, wl.softmax_scale, out=sl["o"],
+                                     workspace=sl["ws"], stream=stream)
+                done = torch.cuda.Event()
+                done.record(stream)
+                ev_done[i & 1] = done
+                if i + 1 < n_steps:
+                    upload(i + 1)
+                with torch.cuda.stream(down):
+                    down.wait_event(done)
+                    sl["ho"].copy_(sl["o"], non_blocking=True)
+                    out = torch.cuda.Event()
+                    out.record(down)
+                    ev_out[i & 1] = out
+            stream.wait_stream(down)
+            stream.wait_stream(up)
 
-    start = torch.cuda.Event()
-    start.record(stream)
-    pipelined(2, start)                 # warm-up of the pipeline
-    torch.cuda.synchronize()
-    barrier()
-    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    p0.record(stream)
-    pipelined(args.steps, p0)
-    p1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    for sl in slots:
-        if h3.device_status_t(sl["ws"]) != h3.H3_OK:
-            raise RuntimeError("device status not ok after the end-to-end steps")
-    e2e_ms = max_over_ranks(p0.elapsed_time(p1), world, dev)
-    e2e_value = job_tflops(world, flops_step, args.steps, e2e_ms)
-    e2e_serial_value = job_tflops(world, flops_step, args.steps, e2e_serial_ms)
+        start = torch.cuda.Event()
+        start.record(stream)
+        pipelined(2, start)                 # warm-up of the pipeline
+        torch.cuda.synchronize()
+        barrier()
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record(stream)
+        pipelined(args.steps, p0)
+        p1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        for sl in slots:
+            if h3.device_status_t(sl["ws"]) != h3.H3_OK:
+                raise RuntimeError("device status not ok after the end-to-end steps")
+        e2e_ms = max_over_ranks(p0.elapsed_time(p1), world, dev)
+        e2e_value = job_tflops(world, flops_step, args.steps, e2e_ms)
+        e2e_serial_value = job_tflops(world, flops_step, args.steps, e2e_serial_ms)
+        return e2e_value, e2e_serial_value, e2e_ms, e2e_serial_ms, h2d, d2h
+
+    e2e_res = None if args.no_e2e else run_e2e()
 
     peaks = measured_peaks()
     achieved = flops_step / (mean_step_ms * 1e-3) / 1e12
@@ -431,15 +436,17 @@ def run_ours(args, wl, rank, world, local_rank):
                      "peak_kind": f"bf16 dense, burst ({peaks['source']})",
                      "traffic": recorded_traffic(wl.name),
                      "kernel": "attn_fwd_kernel<128> (step = k rotary pass + attention kernel)"},
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms / args.steps,
-                "mode": "pipelined: step i+1's host->device copy and step i-1's "
-                        "device->host copy overlap step i's kernels (two device slots)",
-                "serial_value": e2e_serial_value,
-                "serial_ms_per_step": e2e_serial_ms / args.steps},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
     }
+    if e2e_res is not None:
+        e2e_value, e2e_serial_value, e2e_ms, e2e_serial_ms, h2d, d2h = e2e_res
+        line["e2e"] = {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                       "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms / args.steps,
+                       "mode": "pipelined: step i+1's host->device copy and step i-1's "
+                               "device->host copy overlap step i's kernels (two device slots)",
+                       "serial_value": e2e_serial_value,
+                       "serial_ms_per_step": e2e_serial_ms / args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle  # CPU baseline leg only
         def host_bits(t):
@@ -753,6 +760,82 @@ def run_qkv_attend(args, wl, rank, world, local_rank):
     return 0
 
 
+def run_ulysses(args, wl, rank, world, local_rank):
+    """The Ulysses head-sharded path ("MiniMax H3" vLLM-Omni recipe, section
+    "Four GPUs: throughput-oriented combined service": --usp 4): one packed
+    workload is split into contiguous token shards, one per rank; each step
+    runs ulysses_attention (all-to-all sequence -> heads over NCCL, the fused
+    RoPE + varlen attention on H/P heads of the whole sequence, all-to-all
+    back). Strong scaling: the job processes one workload per step whatever
+    the number of ranks. With one rank the wrapper is the kernel call."""
+    import torch
+    import torch.distributed as dist
+
+    import audio_diffusion_transformer_h3_b200 as h3
+    from audio_diffusion_transformer_h3_b200.ulysses import ulysses_attention
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    N, H, D = wl.n_tokens, wl.heads, wl.head_dim
+    if N % world or H % world:
+        raise ValueError(f"{N} tokens and {H} heads must split over {world} ranks")
+    q, k, v = synth.draw_qkv(wl)
+    pos, cu = h3.h3_build_positions(wl.segments)
+    lo, hi = rank * N // world, (rank + 1) * N // world
+
+    def shard(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits[lo:hi]).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    dq, dk, dv = shard(q), shard(k), shard(v)
+    del q, k, v
+    dpos, dcu = torch.from_numpy(pos).to(dev), torch.from_numpy(cu).to(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return ulysses_attention(dq, dk, dv, dcu, wl.max_seqlen, dpos, wl.split, wl.theta,
+                                 wl.softmax_scale)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    visible = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    smi_id = visible[local_rank] if local_rank < len(visible) else str(local_rank)
+    with ClockSampler(smi_id) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    value = wl.flops() * args.steps / (total_ms * 1e-3) / 1e12
+    peaks = measured_peaks()
+    per_gpu = value / world
+    exchanged = 4 * N * H * D * 2 * (world - 1) / world ** 2 if world > 1 else 0
+    line = {"metric": METRIC + " (Ulysses head-sharded, one workload across the ranks)",
+            "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded bf16 ~N(0,1) q/k/v, fp32 positions)",
+            "config": {**workload_config(wl), "parallelism": f"ulysses{world}"},
+            "roofline": {"bound": "tensor", "achieved": per_gpu, "peak": peaks["bf16"],
+                         "unit": "TFLOP/s per GPU", "frac": per_gpu / peaks["bf16"],
+                         "peak_kind": f"bf16 dense, burst ({peaks['source']})"},
+            "all_to_all_bytes_per_rank_per_step": exchanged,
+            "gpu_launches": 2 * args.steps, "clocks": clk.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -763,12 +846,16 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end leg (profiling runs: less device memory)")
     ap.add_argument("--skip-threshold", type=float, default=None,
                     help="time the skip-softmax variant on frame-group inputs instead")
     ap.add_argument("--sage", action="store_true",
                     help="time the SAGE-style FP8 variant instead")
     ap.add_argument("--qkv-proj", action="store_true",
                     help="time the QKV projection with the fused RoPE epilogue instead")
+    ap.add_argument("--ulysses", action="store_true",
+                    help="time the Ulysses head-sharded path (one workload over the ranks)")
     ap.add_argument("--attend", action="store_true",
                     help="with --qkv-proj: time the projection chained into the attention")
     args = ap.parse_args()
@@ -800,6 +887,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.ulysses:
+            return run_ulysses(args, wl, rank, world, local_rank)
         return run_ours(args, wl, rank, world, local_rank)
     finally:
         if world > 1:
