@@ -67,14 +67,16 @@ def ulysses_attention(q, k, v, cu_seqlens, max_seqlen: int, pos=None, split=None
     q, k, v: this rank's [N/P, H, D] token shard (rank r holds tokens
     [r N/P, (r+1) N/P) of the packed sequence). cu_seqlens [nseg+1] and pos
     [N, 3] are global (the same on every rank). Requires N and H divisible by
-    the group size. ``attn`` defaults to the CUDA kernel
+    the group size (one rank when no process group is initialised). ``attn``
+    defaults to the CUDA kernel
     (``varlen_attn_fwd_t``); it is called as
     ``attn(q, k, v, cu_seqlens, max_seqlen, pos, split, theta, softmax_scale,
     return_lse=...)`` on [N, H/P, D] tensors. Returns O [N/P, H, D] (and LSE
     [H, N/P] if asked).
     """
     import torch.distributed as dist
-    world = dist.get_world_size(group)
+    # without an initialised process group the caller is a single rank
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
     n_local, H, D = q.shape
     if H % world:
         raise ValueError(f"{H} heads do not split over {world} ranks")

@@ -130,3 +130,17 @@ def test_two_gloo_ranks_bench_plumbing_and_ulysses_wrapper():
     assert not alive, "a rank did not finish"
     assert not msgs, "\n".join(msgs)
     assert all(p.exitcode == 0 for p in procs)
+
+
+def test_ulysses_without_a_process_group_is_one_rank():
+    # no torch.distributed group: the wrapper is the attention call itself
+    import torch
+    import oracle
+    import synth
+    from audio_diffusion_transformer_h3_b200.ulysses import ulysses_attention
+    q, k, v, pos, cu = synth.draw_random_case([30, 34], 2, 8, seed=78, pos_range=16.0)
+    Q, K, V = (torch.from_numpy(oracle.bf16_bits_to_f64(x)) for x in (q, k, v))
+    out = ulysses_attention(Q, K, V, torch.from_numpy(cu), 34, torch.from_numpy(pos), (2, 4, 2),
+                            1e4, 0.3, attn=_oracle_attn)
+    O, _ = oracle.attention_ref(Q.numpy(), K.numpy(), V.numpy(), cu, 0.3, pos, (2, 4, 2), 1e4)
+    np.testing.assert_allclose(out.numpy(), O, rtol=0, atol=0)
