@@ -26,20 +26,20 @@
 //               period apart so that one tile's products run while the other
 //               exponentiates. A quarter of the exponentials run as a cubic
 //               on the FMA pipe.
-//   warps 8, 9  MMA issuers, warp 8 + t for query tile t (the whole warp
-//               runs the schedule, one elected lane issues): S_t = Q_t K_j^T
-//               (A, B from shared memory) and O_t += P_t V_j (A = P from
-//               TMEM, B = V from shared memory). The score tile is computed
-//               in two 64-key halves: the half whose TMEM columns P_t(j) does
-//               not use (keys 64..127) is issued as soon as the softmax has
-//               read S_t(j) into registers, the other half after PV_t(j);
-//               PV_t(j) runs in two halves as the halves of P_t(j) arrive,
-//               so after the softmax releases the last half only PV over keys
-//               64..127 and the low half of S_t(j+1) remain on the tile's
-//               dependency chain.
+//   warp 8      MMA issuer for both query tiles (the whole warp runs the
+//               schedule, one elected lane issues): S_t = Q_t K_j^T (A, B
+//               from shared memory) and O_t += P_t V_j (A = P from TMEM, B =
+//               V from shared memory), in the order the turns produce them:
+//               per key tile j, tile 0 then tile 1, each as PV over keys
+//               0..63 as soon as the first half of P_t(j) is in TMEM, then
+//               PV over keys 64..127 and S_t(j+1) when the second half
+//               arrives. One issuing warp keeps the MMA instructions, which
+//               take issue slots from the softmax warps of the same
+//               sub-partition, on one sub-partition.
 //   warp 10     TMA producer (converged warp, elected lane issues): Q0/Q1
 //               once, then K_j and V_j through a two-stage ring
-//               (128B-swizzled boxes of 128 rows x 64 cols); warp 11 idles.
+//               (128B-swizzled boxes of 128 rows x 64 cols); warps 9 and 11
+//               idle.
 // The producer warpgroup gives up registers (setmaxnreg) to the two softmax
 // warpgroups.
 // TMEM: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D) fp32
@@ -111,13 +111,13 @@ struct AttnCfg {
                   "register split exceeds the launch allocation");
 };
 
-// Barrier slots (uint64 each) at OFF_BAR.
-// S_t full (both halves), S_t consumed (read into registers: its columns may
-// be overwritten), first and second half of P_t written, O_t final.
+// Barrier slots (uint64 each) at OFF_BAR: per query tile t, S_t full, the
+// two halves of P_t written, O_t final; per SM sub-partition the two
+// exponential turns (B_TURN + q: tile 1 has finished key tile j there;
+// B_TURN + 4 + q: tile 0 has).
 enum : int {
     B_QFULL = 0, B_QREADY = 1, B_KFULL = 2, B_KEMPTY = 4, B_VFULL = 6, B_VEMPTY = 8,
-    B_SFULL = 10, B_SCONS = 12, B_P1 = 14, B_P2 = 16, B_OFULL = 18, B_DRAIN = 20, B_TURN = 22,
-    B_COUNT = 30
+    B_SFULL = 10, B_P1 = 12, B_P2 = 14, B_OFULL = 16, B_DRAIN = 18, B_TURN = 19, B_COUNT = 27
 };
 
 __device__ __forceinline__ void raise_abort(volatile int *abort, int *status) {
@@ -199,13 +199,11 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&bars[B_VFULL + s], 1);
             mbar_init(&bars[B_VEMPTY + s], 2);   // one commit per query tile
             mbar_init(&bars[B_SFULL + s], 1);
-            mbar_init(&bars[B_SCONS + s], 4);    // one arrival per softmax warp
             mbar_init(&bars[B_P1 + s], 4);
             mbar_init(&bars[B_P2 + s], 4);
             mbar_init(&bars[B_OFULL + s], 1);
         }
         mbar_init(&bars[B_DRAIN], 1);
-        mbar_init(&bars[B_DRAIN + 1], 1);
         for (int i = 0; i < 8; ++i) mbar_init(&bars[B_TURN + i], 1);
         *abort = 0;
         for (int i = 0; i < 8; ++i) skipword[i] = 0;
@@ -276,50 +274,37 @@ __global__ void __launch_bounds__(384, 1)
                 mbar_wait(&bars[B_VFULL + (j & 1)], (j >> 1) & 1, nullptr);
         }
         __syncwarp();
-    } else if (warp >= 8) {
-        // ============================ MMA issuers =============================
-        // Warp 8 issues every MMA of query tile 0, warp 9 every MMA of tile 1,
-        // each in its tile's order and waiting (bounded, suspending) on that
-        // tile's barriers only. The whole warp runs the schedule so that it
-        // stays converged; only the elected lane issues the MMAs and commits.
-        // tcgen05.commit tracks the MMAs of the committing thread, so each
-        // warp's commits cover its own tile; the K and V slots are released
-        // by one commit from each warp.
+    } else if (warp == 9) {
         reg_dealloc<C::REGS_PRODUCER>();
-        const int t = warp - 8;
+    } else if (warp == 8) {
+        reg_dealloc<C::REGS_PRODUCER>();
         const uint32_t leader = elect_one();
         constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
-        constexpr uint32_t IDESC_SH = idesc_bf16_f32(128, 64, false, false);
         constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
-        const uint32_t sQ = smem_u32(smem + C::OFF_Q) + t * C::TILE_BYTES;
+        const uint32_t sQ0 = smem_u32(smem + C::OFF_Q);
         const uint32_t sK = smem_u32(smem + C::OFF_K);
         const uint32_t sV = smem_u32(smem + C::OFF_V);
-        const uint32_t colS = tmem + (t ? C::COL_S1 : C::COL_S0);
-        const uint32_t colO = tmem + (t ? C::COL_O1 : C::COL_O0);
-        // S_t, or its 64-key half: key rows [r0, r0 + n) of the K tile in
-        // slot ks into TMEM columns [r0, r0 + n) of S_t
-        const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);
+        const uint64_t dQ = sdesc_sw128(sQ0, 16, 1024);
         const uint64_t dK = sdesc_sw128(sK, 16, 1024);
         const uint64_t dV = sdesc_sw128(sV, C::BOX_BYTES, 1024);
-        auto issue_s = [&](int ks, int r0, int n) {
-            const uint64_t dk = dK + static_cast<uint64_t>((ks * C::TILE_BYTES + r0 * 128) >> 4);
+        auto issue_s = [&](int t, int ks) {
+            const uint32_t colS = tmem + (t ? C::COL_S1 : C::COL_S0);
+            const uint64_t dq = dQ + static_cast<uint64_t>((t * C::TILE_BYTES) >> 4);
+            const uint64_t dk = dK + static_cast<uint64_t>((ks * C::TILE_BYTES) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t off = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
-                umma_ss_w(colS + r0, dQ + off, dk + off, n == 128 ? IDESC_S : IDESC_SH,
-                          kk > 0 ? 1u : 0u, leader);
+                umma_ss_w(colS, dq + off, dk + off, IDESC_S, kk > 0 ? 1u : 0u, leader);
             }
         };
-        // O_t += P_t V_j over keys [16 k0, 16 k1) of the tile
-        auto issue_pv = [&](int j, int k0, int k1) {
+        auto issue_pv = [&](int t, int j, int k0, int k1) {
+            const uint32_t colS = tmem + (t ? C::COL_S1 : C::COL_S0);
+            const uint32_t colO = tmem + (t ? C::COL_O1 : C::COL_O0);
             const uint64_t dv = dV + static_cast<uint64_t>(((j & 1) * C::TILE_BYTES) >> 4);
 #pragma unroll
-            for (int kk = k0; kk < k1; ++kk) {
-                // V tile [128 keys][D] is MN-major for B: 8 key rows at 128 B,
-                // groups of 8 rows at SBO = 1024 B, 64-col boxes at LBO.
+            for (int kk = k0; kk < k1; ++kk)
                 umma_ts_w(colO, colS + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4),
                           IDESC_O, (j > 0 || kk > 0) ? 1u : 0u, leader);
-            }
         };
         auto wait = [&](int bar, uint32_t parity) {
             return __all_sync(0xffffffffu, mbar_wait(&bars[bar], parity, abort));
@@ -327,48 +312,47 @@ __global__ void __launch_bounds__(384, 1)
         bool ok = wait(B_QREADY, 0) && wait(B_KFULL, 0);
         if (ok) {
             tc_fence_after();
-            issue_s(0, 0, 128);
-            umma_commit_w(&bars[B_SFULL + t], leader);
-            umma_commit_w(&bars[B_KEMPTY], leader);
+            for (int t = 0; t < 2; ++t) {
+                issue_s(t, 0);
+                umma_commit_w(&bars[B_SFULL + t], leader);
+                umma_commit_w(&bars[B_KEMPTY], leader);
+            }
         }
         for (int j = 0; ok && j < n_kv; ++j) {
             const bool more = j + 1 < n_kv;
             const int ks = (j + 1) & 1;
-            // keys 64..127 of the next tile into the columns P_t(j) leaves free,
-            // as soon as the softmax holds S_t(j) in registers
-            if (more) {
-                ok = wait(B_SCONS + t, j & 1) && wait(B_KFULL + ks, ((j + 1) >> 1) & 1);
+            for (int t = 0; ok && t < 2; ++t) {
+                ok = wait(B_P1 + t, j & 1) && wait(B_VFULL + (j & 1), (j >> 1) & 1);
                 if (!ok) break;
                 tc_fence_after();
-                issue_s(ks, 64, 64);
-            }
-            ok = wait(B_P1 + t, j & 1) && wait(B_VFULL + (j & 1), (j >> 1) & 1);
-            if (!ok) break;
-            tc_fence_after();
-            bool skip_pv = false;
-            if constexpr (SKIP) {
-                const uint32_t tag = static_cast<uint32_t>(j + 1);
-                skip_pv = skipword[t * 4 + 0] == tag && skipword[t * 4 + 1] == tag &&
-                          skipword[t * 4 + 2] == tag && skipword[t * 4 + 3] == tag;
-            }
-            if (!skip_pv) issue_pv(j, 0, C::BN / 32);
-            ok = wait(B_P2 + t, j & 1);
-            if (!ok) break;
-            tc_fence_after();
-            if (!skip_pv) issue_pv(j, C::BN / 32, C::BN / 16);
-            umma_commit_w(&bars[B_VEMPTY + (j & 1)], leader);
-            if (more) {
-                issue_s(ks, 0, 64);
-                umma_commit_w(&bars[B_SFULL + t], leader);
-                umma_commit_w(&bars[B_KEMPTY + ks], leader);
-            } else {
-                umma_commit_w(&bars[B_OFULL + t], leader);
+                bool skip_pv = false;
+                if constexpr (SKIP) {
+                    const uint32_t tag = static_cast<uint32_t>(j + 1);
+                    skip_pv = skipword[t * 4 + 0] == tag && skipword[t * 4 + 1] == tag &&
+                              skipword[t * 4 + 2] == tag && skipword[t * 4 + 3] == tag;
+                }
+                if (!skip_pv) issue_pv(t, j, 0, C::BN / 32);
+                ok = wait(B_P2 + t, j & 1);
+                if (!ok) break;
+                tc_fence_after();
+                if (!skip_pv) issue_pv(t, j, C::BN / 32, C::BN / 16);
+                umma_commit_w(&bars[B_VEMPTY + (j & 1)], leader);
+                if (more) {
+                    ok = wait(B_KFULL + ks, ((j + 1) >> 1) & 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s(t, ks);
+                    umma_commit_w(&bars[B_SFULL + t], leader);
+                    umma_commit_w(&bars[B_KEMPTY + ks], leader);
+                } else {
+                    umma_commit_w(&bars[B_OFULL + t], leader);
+                }
             }
         }
         if (!ok) {
             if (leader) raise_abort(abort, p.status);
-            umma_commit_w(&bars[B_DRAIN + t], leader);  // completes once this warp's MMAs are done
-            mbar_wait(&bars[B_DRAIN + t], 0, nullptr);
+            umma_commit_w(&bars[B_DRAIN], leader);
+            mbar_wait(&bars[B_DRAIN], 0, nullptr);
         }
         __syncwarp();
     } else {
@@ -437,11 +421,6 @@ __global__ void __launch_bounds__(384, 1)
             tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
             tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
             tmem_wait_ld();
-            // S_t(j) is in registers: the MMA warp may now overwrite its columns
-            // 64..127 with the next tile's scores
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_SCONS + t]);
             const int kv_valid = seg_end - (seg_start + j * C::BN);
             if (kv_valid < C::BN) {
 #pragma unroll
