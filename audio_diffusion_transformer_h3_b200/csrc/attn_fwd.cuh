@@ -24,8 +24,8 @@
 //               0 exponentiates key tile j, then tile 1 key tile j, then tile
 //               0 key tile j + 1, ...), which keeps the two tiles half a
 //               period apart so that one tile's products run while the other
-//               exponentiates. A quarter of the exponentials run as a cubic
-//               on the FMA pipe.
+//               exponentiates. Three eighths of the exponentials run as a
+//               cubic on the FMA pipe.
 //   warp 8      MMA issuer for both query tiles (the whole warp runs the
 //               schedule, one elected lane issues): S_t = Q_t K_j^T (A, B
 //               from shared memory) and O_t += P_t V_j (A = P from TMEM, B =
@@ -57,11 +57,11 @@
 #include "sm100.cuh"
 
 // Key pairs out of every eight whose exponentials run on the FMA pipe
-// (exp2_fma2, a cubic on the FMA and integer pipes) instead of MUFU: a
-// quarter of them, which shortens each softmax warp's exponential phase
-// (measured: 2 of 8 ahead of 0 and 1 of 8, level with 3 of 8).
+// (exp2_fma2, a cubic on the FMA and integer pipes) instead of MUFU: three of
+// eight, which shortens each softmax warp's exponential phase (measured: 3 of
+// 8 ahead of 0, 1 and 2 of 8; 4 of 8 slower).
 #ifndef H3_FMA_EXP2_PAIRS
-#define H3_FMA_EXP2_PAIRS 2
+#define H3_FMA_EXP2_PAIRS 3
 #endif
 
 namespace h3 {
@@ -427,12 +427,16 @@ __global__ void __launch_bounds__(384, 1)
                 for (int c = 0; c < 128; ++c)
                     if (c >= kv_valid) s[c] = __float_as_uint(-INFINITY);
             }
-            // row max over 128 keys in 8 independent chains (ALU throughput, not latency)
+            // row max over 128 keys in 8 independent chains of three-input max
+            // (ALU throughput, not latency)
             float mq[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) mq[i] = __uint_as_float(s[i]);
 #pragma unroll
-            for (int c = 8; c < 128; ++c) mq[c & 7] = fmaxf(mq[c & 7], __uint_as_float(s[c]));
+            for (int c = 8; c < 128; c += 16)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    mq[i] = fmax3(mq[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 8 + i]));
             const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
                                    fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
             const float m_new = mx * sl2;
