@@ -130,7 +130,6 @@ h3_status device_info(DeviceInfo **out) {
                              attn_regs_cover_split(h3::attn_fwd_kernel<128, true>, 128) &&
                              attn_regs_cover_split(h3::attn_fwd_kernel<64, false>, 64) &&
                              attn_regs_cover_split(h3::attn_fwd_kernel<64, true>, 64);
-
         }
         d.ready = true;
     }
