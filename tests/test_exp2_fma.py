@@ -72,3 +72,21 @@ def test_monotone_and_nonnegative_including_clamp():
     # non-decreasing up to the polynomial's relative error at the interval joints
     d = np.diff(y.astype(np.float64)) / y[1:].astype(np.float64).clip(1e-300)
     assert d.min() >= -2e-4
+
+
+def test_packed_form_uses_the_same_method_and_constants():
+    # exp2_fma2 (two lanes in f32x2 registers, used by the dense softmax) takes the
+    # same steps as exp2_fma: the clamp, the shift pair, f = x - rint(x) (as
+    # fma(rint(x), -1, x), exact), the cubic by Horner with the same coefficients,
+    # and j added to the exponent field
+    text = open(SRC).read()
+    body = text[text.index("void exp2_fma2("):]
+    body = body[:body.index("\n}\n")]
+    (c0, c1, c2, c3), shift, clamp = _coeffs()
+    consts = [np.float32(v) for v in re.findall(r'"f"\(([-0-9.eE]+)f\)', body)]
+    assert consts == [shift, -shift, np.float32(-1.0), c0, c1, c2, c3], consts
+    assert body.count(f"fmaxf(x0, {clamp:.1f}f)") == 1 and body.count(f"fmaxf(x1, {clamp:.1f}f)") == 1
+    steps = re.findall(r"(add|fma)\.rn\.f32x2 (\w+), (\w+), (\w+)(?:, (\w+))?;", body)
+    assert [s[:3] for s in steps] == [("add", "ta", "xa"), ("add", "ra", "ta"), ("fma", "fa", "ra"),
+                                      ("fma", "pa", "c3"), ("fma", "pa", "pa"), ("fma", "pa", "pa")]
+    assert body.count("* 8388608u +") == 2
