@@ -15,8 +15,10 @@
 //   more than 2 (log2 units), so 2^(x - m) <= 4; P8 = e4m3(112 * 2^(x - m))
 //   (<= 448); the row sum l adds the unquantised 112 * 2^(x - m);
 //   O = s_v * (P8 V8) / l. Exponentials: three quarters on MUFU
-//   (ex2.approx), one quarter on the FMA pipe (exp2_fma, relative error
-//   below 2e-4), which shares the load between the two pipes.
+//   (ex2.approx), one quarter on the FMA pipe (exp2_fma / exp2_fma2,
+//   relative error below 2e-4), which shares the load between the two pipes;
+//   the scale-and-shift of the scores and the row sums run as packed f32x2
+//   FFMA/FADD.
 // e4m3 conversions round to nearest even and saturate to +-448
 // (cvt.rn.satfinite).
 //
@@ -558,19 +560,36 @@ __global__ void __launch_bounds__(320, 1)
                     pk[w] = e4m3x4(pv[0], pv[1], pv[2], pv[3]);
                 }
             } else {
+                // packed f32x2 arithmetic: the scale-and-shift of two scores of one
+                // 16-key block in one FFMA2, the row sum in FADD2
+                const uint64_t n2 = f2_splat(nm);
+                uint64_t acc0 = 0, acc1 = 0;
 #pragma unroll
                 for (int w = 0; w < 32; ++w) {
-                    float pv[4];
+                    const uint64_t c2 = f2_splat(cb[w >> 2]);
+                    float y[4], pv[4];
+                    ffma2(y[0], y[1], __uint_as_float(s[4 * w]), __uint_as_float(s[4 * w + 1]), c2, n2);
+                    ffma2(y[2], y[3], __uint_as_float(s[4 * w + 2]), __uint_as_float(s[4 * w + 3]), c2,
+                          n2);
+                    // words 6 and 7 of every 8 on the FMA pipe, the rest on MUFU
+                    if ((w & 7) >= 6) {
+                        exp2_fma2(pv[0], pv[1], y[0], y[1]);
+                        exp2_fma2(pv[2], pv[3], y[2], y[3]);
+                    } else {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int c = 4 * w + i;
-                        const float y = fmaf(__uint_as_float(s[c]), cb[c >> 4], nm);
-                        // words 6 and 7 of every 8 on the FMA pipe, the rest on MUFU
-                        pv[i] = (w & 7) >= 6 ? exp2_fma(y) : ex2_approx(y);
+                        for (int i = 0; i < 4; ++i) pv[i] = ex2_approx(y[i]);
                     }
-                    lq[w & 3] += (pv[0] + pv[1]) + (pv[2] + pv[3]);
+                    if (w & 1) {
+                        fadd2(acc1, pv[0], pv[1]);
+                        fadd2(acc1, pv[2], pv[3]);
+                    } else {
+                        fadd2(acc0, pv[0], pv[1]);
+                        fadd2(acc0, pv[2], pv[3]);
+                    }
                     pk[w] = e4m3x4(pv[0], pv[1], pv[2], pv[3]);
                 }
+                lq[0] += f2_sum(acc0);
+                lq[1] += f2_sum(acc1);
             }
             l += (lq[0] + lq[1]) + (lq[2] + lq[3]);
             if (__any_sync(0xffffffffu, need)) {
