@@ -8,7 +8,9 @@ runs ``varlen_attn_fwd_t`` on the GPU for its head group, and the second
 all-to-all returns its tokens (gloo all-to-all carries bf16 tensors). The kernels of the two ranks do not wait on
 each other (each launch is independent; the exchange is on the host). Each
 rank's O and LSE must match the whole-sequence float64 oracle within the
-path's tolerance (max |d| <= 2e-2, mean |d| <= 2e-3; LSE within 1e-2).
+path's tolerance (max |d| <= 2e-2, mean |d| <= 2e-3; LSE within 1e-2); with
+the SAGE-style FP8 kernel as the attention step, each rank matches the
+whole-sequence SAGE oracle within the same tolerance.
 """
 
 import math
@@ -38,6 +40,19 @@ def _gpu_attn(q, k, v, cu, max_seqlen, pos, split, theta, scale, return_lse=Fals
     o, lse = h3.varlen_attn_fwd_t(dq, dk, dv, cu.cuda(), max_seqlen,
                                   None if pos is None else pos.cuda(), split, theta, scale,
                                   return_lse=True)
+    torch.cuda.synchronize()
+    o = o.cpu()
+    return (o, lse.cpu()) if return_lse else o
+
+
+def _gpu_sage_attn(q, k, v, cu, max_seqlen, pos, split, theta, scale, return_lse=False):
+    """The SAGE-style FP8 attention step of the wrapper on the GPU."""
+    import torch
+    import audio_diffusion_transformer_h3_b200 as h3
+    dq, dk, dv = (x.cuda() for x in (q, k, v))
+    o, lse = h3.varlen_attn_fwd_sage_t(dq, dk, dv, cu.cuda(), max_seqlen,
+                                       None if pos is None else pos.cuda(), split, theta, scale,
+                                       return_lse=True)
     torch.cuda.synchronize()
     o = o.cpu()
     return (o, lse.cpu()) if return_lse else o
@@ -80,6 +95,16 @@ def _worker(rank, world, port, root, errors):
         assert got.shape == (hi - lo, H, D) and lse.shape == (H, hi - lo)
         assert_close_bf16(got, O[lo:hi], f"ulysses rank {rank}")
         np.testing.assert_allclose(lse.numpy(), L[:, lo:hi], rtol=0, atol=1e-2)
+        # the SAGE-style FP8 kernel quantises per head (Q per token, K per 16-key
+        # block from the segment start, V per segment and channel), so the head
+        # split reproduces the whole-sequence SAGE reading
+        out, lse = ulysses_attention(shard(q), shard(k), shard(v), torch.from_numpy(cu),
+                                     max(seg), torch.from_numpy(pos), split, 1e4, scale,
+                                     attn=_gpu_sage_attn, return_lse=True)
+        Os, Ls = oracle.sage_attention_ref(q, k, v, cu, scale, pos, split, 1e4)
+        assert_close_bf16(out.float().numpy().astype(np.float64), Os[lo:hi],
+                          f"ulysses sage rank {rank}")
+        np.testing.assert_allclose(lse.numpy(), Ls[:, lo:hi], rtol=0, atol=1e-2)
         dist.barrier()
     except Exception as e:  # reported to the parent
         import traceback
