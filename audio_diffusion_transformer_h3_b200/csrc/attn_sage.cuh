@@ -28,8 +28,11 @@
 //   sage_quant_kernel   RoPE + quantisation of q, k, v into e4m3 codes and
 //                       scales; one CTA per 16-token block (all heads, the
 //                       block's rotary table computed once), lane = 4 channels;
-//   attn_sage_kernel    the attention kernel of attn_fwd.cuh in FP8: the same
-//                       warp roles, barriers and TMEM plan, tcgen05.mma
+//   attn_sage_kernel    the attention kernel of attn_fwd.cuh in FP8, with its
+//                       earlier schedule (one MMA warp, the two softmax
+//                       warpgroups free-running, P released at once; 384
+//                       threads, setmaxnreg moving registers to the softmax
+//                       warpgroups) and TMEM plan, tcgen05.mma
 //                       kind::f8f6f4 for S = Q8 K8^T (A, B K-major in shared
 //                       memory) and O += P8 V8 (A = P8 from TMEM, four codes per
 //                       32-bit column; B = V8 MN-major), 16 KB tiles in a
@@ -299,7 +302,15 @@ struct SageCfg {
     static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
     static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 384;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr int THREADS = 320;
+    static constexpr int THREADS = 384;
+    // registers per thread: 168 at launch; the producer warpgroup (MMA, TMA
+    // and two idle warps) drops to 56 and the softmax warpgroups rise to 224
+    // (2 * 128 * 224 + 128 * 56 = 384 * 168)
+    static constexpr int REGS_LAUNCH = 168;
+    static constexpr int REGS_SOFTMAX = 224;
+    static constexpr int REGS_PRODUCER = 56;
+    static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_PRODUCER <= THREADS * REGS_LAUNCH,
+                  "register split exceeds the launch allocation");
 };
 
 enum : int {
@@ -307,7 +318,7 @@ enum : int {
     SB_SFULL = 13, SB_PFULL = 15, SB_OFULL = 17, SB_DRAIN = 19, SB_COUNT = 20
 };
 
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_sage_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const SageAttnParams p) {
@@ -374,8 +385,11 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 9) {
+    if (warp >= 10) {
+        reg_dealloc<C::REGS_PRODUCER>();   // idle warps of the producer warpgroup
+    } else if (warp == 9) {
         // ============================ TMA producer ============================
+        reg_dealloc<C::REGS_PRODUCER>();
         const uint32_t leader = elect_one();
         if (leader) {
             mbar_arrive_expect_tx(&bars[SB_QFULL], 2 * C::TILE_BYTES);
@@ -419,6 +433,7 @@ __global__ void __launch_bounds__(320, 1)
         __syncwarp();
     } else if (warp == 8) {
         // ============================ MMA issuer ==============================
+        reg_dealloc<C::REGS_PRODUCER>();
         const uint32_t leader = elect_one();
         constexpr uint32_t IDESC_S = idesc_e4m3_f32(128, 128, false, false);
         constexpr uint32_t IDESC_O = idesc_e4m3_f32(128, 128, false, true);
@@ -482,6 +497,7 @@ __global__ void __launch_bounds__(320, 1)
         __syncwarp();
     } else {
         // ============================ softmax / epilogue ======================
+        reg_alloc<C::REGS_SOFTMAX>();
         const int t = warp >> 2;
         const int r = tid & 127;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;

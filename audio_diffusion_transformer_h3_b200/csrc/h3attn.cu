@@ -64,6 +64,7 @@ struct DeviceInfo {
     bool ready = false;
     bool sm100 = false;
     bool attn_regs_ok = false;
+    bool sage_regs_ok = false;
     int sms = 0;
     cudaError_t err = cudaSuccess;
 };
@@ -130,6 +131,11 @@ h3_status device_info(DeviceInfo **out) {
                              attn_regs_cover_split(h3::attn_fwd_kernel<128, true>, 128) &&
                              attn_regs_cover_split(h3::attn_fwd_kernel<64, false>, 64) &&
                              attn_regs_cover_split(h3::attn_fwd_kernel<64, true>, 64);
+            cudaFuncAttributes a{};
+            using S = h3::SageCfg;
+            d.sage_regs_ok = cudaFuncGetAttributes(&a, h3::attn_sage_kernel) == cudaSuccess &&
+                             static_cast<long long>(a.numRegs) * S::THREADS >=
+                                 2LL * 128 * S::REGS_SOFTMAX + 128LL * S::REGS_PRODUCER;
         }
         d.ready = true;
     }
@@ -570,6 +576,7 @@ h3_status h3_varlen_attn_fwd_sage(const void *q, const void *k, const void *v, v
     DeviceInfo *d = nullptr;
     h3_status st = device_info(&d);
     if (st != H3_OK) return st;
+    if (!d->sage_regs_ok) return H3_ERR_UNSUPPORTED;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *status = reinterpret_cast<int *>(ws);
