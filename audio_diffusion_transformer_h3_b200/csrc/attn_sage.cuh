@@ -14,9 +14,11 @@
 //   m: m is raised to the running max only when a tile's max exceeds it by
 //   more than 2 (log2 units), so 2^(x - m) <= 4; P8 = e4m3(112 * 2^(x - m))
 //   (<= 448); the row sum l adds the unquantised 112 * 2^(x - m);
-//   O = s_v * (P8 V8) / l. Exponentials: three quarters on MUFU
-//   (ex2.approx), one quarter on the FMA pipe (exp2_fma / exp2_fma2,
-//   relative error below 2e-4), which shares the load between the two pipes;
+//   O = s_v * (P8 V8) / l. Exponentials: half on MUFU (ex2.approx), half
+//   on the FMA pipe (exp2_fma2_deg2: a degree-2 polynomial, relative error
+//   below 1.8e-3, well inside e4m3's 2^-3 relative spacing of the P codes;
+//   tiles with masked keys use ex2.approx throughout), which shares the load
+//   between the two pipes;
 //   the scale-and-shift of the scores and the row sums run as packed f32x2
 //   FFMA/FADD.
 // e4m3 conversions round to nearest even and saturate to +-448
@@ -277,6 +279,40 @@ __device__ __forceinline__ void umma_f8_ss_w(uint32_t d_tmem, uint64_t a_desc, u
         "@q tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader)
         : "memory");
+}
+
+// 2^x for two lanes on the FMA and integer pipes, for P values that are
+// rounded to e4m3 next: the split of exp2_fma (x = j + f, j = rint(x) by adding
+// and subtracting 1.5 * 2^23, j added to the exponent field) with a degree-2
+// polynomial for 2^f on [-1/2, 1/2] instead of degree 3. Its coefficients
+// minimise the largest relative error (Lawson's iteratively reweighted least
+// squares on a fine grid): below 1.8e-3, against e4m3's relative spacing of
+// 2^-3, so a code moves by at most one step and only when the exact value
+// lies within 1.8e-3 of a rounding boundary. One FFMA2 fewer than exp2_fma2.
+__device__ __forceinline__ void exp2_fma2_deg2(float &y0, float &y1, float x0, float x1) {
+    x0 = fmaxf(x0, -126.0f);
+    x1 = fmaxf(x1, -126.0f);
+    uint32_t t0, t1, p0, p1;
+    asm("{\n\t.reg .b64 xa, ta, ra, fa, pa, sh, nsh, nm1, c0, c1, c2;\n\t"
+        "mov.b64 xa, {%4, %5};\n\t"
+        "mov.b64 sh, {%6, %6};\n\t"
+        "mov.b64 nsh, {%7, %7};\n\t"
+        "mov.b64 nm1, {%8, %8};\n\t"
+        "mov.b64 c0, {%9, %9};\n\t"
+        "mov.b64 c1, {%10, %10};\n\t"
+        "mov.b64 c2, {%11, %11};\n\t"
+        "add.rn.f32x2 ta, xa, sh;\n\t"
+        "add.rn.f32x2 ra, ta, nsh;\n\t"
+        "fma.rn.f32x2 fa, ra, nm1, xa;\n\t"
+        "fma.rn.f32x2 pa, c2, fa, c1;\n\t"
+        "fma.rn.f32x2 pa, pa, fa, c0;\n\t"
+        "mov.b64 {%0, %1}, ta;\n\t"
+        "mov.b64 {%2, %3}, pa;\n\t}"
+        : "=r"(t0), "=r"(t1), "=r"(p0), "=r"(p1)
+        : "f"(x0), "f"(x1), "f"(12582912.0f), "f"(-12582912.0f), "f"(-1.0f),
+          "f"(1.00044296495389f), "f"(0.7034428104994397f), "f"(0.23842570308291403f));
+    y0 = __uint_as_float(t0 * 8388608u + p0);
+    y1 = __uint_as_float(t1 * 8388608u + p1);
 }
 
 __device__ __forceinline__ void umma_f8_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
@@ -587,10 +623,10 @@ __global__ void __launch_bounds__(384, 1)
                     ffma2(y[0], y[1], __uint_as_float(s[4 * w]), __uint_as_float(s[4 * w + 1]), c2, n2);
                     ffma2(y[2], y[3], __uint_as_float(s[4 * w + 2]), __uint_as_float(s[4 * w + 3]), c2,
                           n2);
-                    // words 6 and 7 of every 8 on the FMA pipe, the rest on MUFU
-                    if ((w & 7) >= 6) {
-                        exp2_fma2(pv[0], pv[1], y[0], y[1]);
-                        exp2_fma2(pv[2], pv[3], y[2], y[3]);
+                    // words 4..7 of every 8 on the FMA pipe, the rest on MUFU
+                    if ((w & 7) >= 4) {
+                        exp2_fma2_deg2(pv[0], pv[1], y[0], y[1]);
+                        exp2_fma2_deg2(pv[2], pv[3], y[2], y[3]);
                     } else {
 #pragma unroll
                         for (int i = 0; i < 4; ++i) pv[i] = ex2_approx(y[i]);
