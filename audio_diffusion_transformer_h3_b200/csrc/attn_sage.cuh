@@ -143,7 +143,10 @@ __global__ void __launch_bounds__(256) sage_vamax_kernel(const SageQuantParams p
 // pairs) in shared memory, then warp w quantises heads w, w + 8, ...; lane l
 // holds channels 4l .. 4l+3 (rotary pairs 2l and 2l+1). All 48 row fragments
 // of a (block, head) are loaded before the first store.
-__global__ void __launch_bounds__(256) sage_quant_kernel(const SageQuantParams p) {
+// Two CTAs per SM (at most 128 registers a thread): the second CTA's loads
+// overlap the first one's arithmetic (measured 1.13 against 1.54 ms at 78,408
+// tokens x 48 heads, codes bit-identical).
+__global__ void __launch_bounds__(256, 2) sage_quant_kernel(const SageQuantParams p) {
     __shared__ float4 cs[16][32];   // per token and lane: (cos, sin) of pairs 2l, 2l+1
     const int seg = blockIdx.y, blk = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
